@@ -1,0 +1,466 @@
+"""Benchmark of one absorbed MLA decode step (one layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+                    [--workload NAME] [--num-splits S]
+
+A step is the whole hot path over one batch: mla_absorb_q -> mla_decode ->
+mla_combine (when split) -> mla_up_proj, through the C ABI. The default
+workload is the DeepSeek-V3 decode shape (B=64, H=128, Q=1, Dn=128, Dr=64,
+Vd=128, Ckv=512, Lk=4096, bf16 storage, contiguous cache). Inputs are
+seeded synthetic data resident in HBM before timing; L2 is flushed (a
+256 MiB write) before every timed step, outside the step's events.
+
+Reported (one JSON line from rank 0):
+  value        decode tokens/s over all ranks (B*Q*N / max-over-ranks step time)
+  roofline     the decode kernel (the dominant launch): algorithmic bytes per
+               launch / its mean CUDA-event duration, against measured HBM peak
+  step         whole-step bytes, flops, TB/s, TFLOP/s and fraction of
+               max(bytes/HBM peak, flops/bf16 peak)
+  e2e          the same metric with per-step H2D of q_nope/q_pe from pinned host
+               memory and D2H of the output inside the timed region
+  cpu_baseline the fp64 oracle timed on the host cores on a bounded sample
+
+With N > 1 (torchrun), each rank decodes its own batch of the same shape
+(data-parallel over sequences; no collective on the data path) and the
+step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s and achieved HBM TB/s (% of roofline) per MLA layer, 1×B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def make_workload(name: str, rank: int):
+    from latent_kv_decode_b200 import workloads as wl
+    if name == "dsv3_b64_lk4096":
+        return wl.dsv3(seed=1 + 1000 * rank)
+    if name == "longctx_b4_lk131072":
+        return wl.longctx(seed=3 + 1000 * rank)
+    if name == "ragged_paged_b128_q2":
+        return wl.ragged_paged(seed=2 + 1000 * rank)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def workload_desc(w) -> dict:
+    d = dict(workload=f"{w.name}: B={w.B} H={w.H} Q={w.Q} Dn={w.Dn} Dr={w.Dr} Vd={w.Vd} "
+                      f"Ckv={w.Ckv} Lk={w.Lk}{' ragged paged' if w.block_table is not None else ''}"
+                      f", {w.dtype} storage, fp32 accumulate",
+             B=w.B, H=w.H, Q=w.Q, Lk=w.Lk, Dn=w.Dn, Dr=w.Dr, Vd=w.Vd, Ckv=w.Ckv,
+             cache="paged 64-token pages" if w.block_table is not None else "contiguous",
+             l2="flushed before every timed step (256 MiB write); cache larger than L2")
+    return d
+
+
+def algorithmic(w):
+    """Algorithmic bytes / flops of one step and of the decode launch.
+
+    Decode: every visible cache row once (Ckv+Dr elements), q_lat and q_pe
+    read once, x written once. Step: plus W_UK and W_UV read once, q_nope read,
+    q_lat written and read, x read, out written. Flops: 2*H*Q*(Ckv+Dr) per
+    visible token for the scores and 2*H*Q*Ckv for the aggregation, plus the
+    two projections 2*B*Q*H*Ckv*(Dn+Vd).
+    """
+    es = 4 if w.dtype == "f32" else 2
+    L = w.lens()
+    if w.causal:
+        vis_rows = sum(int(l) - w.Q + 1 + q for l in L for q in range(w.Q)) / w.Q
+    else:
+        vis_rows = float(L.sum())
+    rows_read = float(L.sum())
+    HQ = w.H * w.Q
+    dec_bytes = rows_read * (w.Ckv + w.Dr) * es + w.B * HQ * (w.Ckv + w.Dr) * es + w.B * HQ * w.Ckv * es
+    dec_flops = vis_rows * w.Q * w.H * 2 * ((w.Ckv + w.Dr) + w.Ckv)
+    proj_bytes = (w.H * (w.Dn + w.Vd) * w.Ckv * es + w.B * HQ * w.Dn * es + w.B * HQ * w.Ckv * es
+                  + w.B * HQ * w.Ckv * es + w.B * HQ * w.Vd * es)
+    proj_flops = 2 * w.B * HQ * w.Ckv * (w.Dn + w.Vd)
+    return dict(decode_bytes=dec_bytes, decode_flops=dec_flops,
+                step_bytes=dec_bytes + proj_bytes, step_flops=dec_flops + proj_flops)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "latent_kv_decode_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
+    m_bytes = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", txt)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    from latent_kv_decode_b200 import ops
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.workload, rank)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def up(a, dtype=dt):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).to(dev)
+
+    q_nope, q_pe, wkv_b = up(w.q_nope), up(w.q_pe), up(w.wkv_b)
+    if w.block_table is not None:
+        kv, pe = up(w.kv_pool), up(w.pe_pool)
+        bt = torch.from_numpy(w.block_table).to(dev)
+    else:
+        kv, pe = up(w.kv_cache), up(w.pe_cache)
+        bt = None
+    seq_lens = torch.from_numpy(w.seq_lens).to(dev) if w.seq_lens is not None else None
+    B, H, Q = w.B, w.H, w.Q
+    q_lat = torch.empty((B, H, Q, w.Ckv), dtype=dt, device=dev)
+    out = torch.empty((B, H, Q, w.Vd), dtype=dt, device=dev)
+    call = ops.make_decode_args(q_lat, q_pe, kv, pe, w.softmax_scale, seq_lens=seq_lens,
+                                block_table=bt, page_size=w.page_size, causal=w.causal,
+                                num_splits=args.num_splits,
+                                Lk=w.Lk if bt is None else None)
+    need = ops.workspace_bytes(call)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    split = call.num_splits > 1
+    launches_per_step = 3 + (1 if split else 0)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ops.mla_absorb_q(q_nope, wkv_b, q_lat, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        ops.launch_decode(call, ws, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        if split:
+            ops.mla_combine(call, stream=stream)
+        if evs:
+            evs[3].record(stream)
+        ops.mla_up_proj(call.x, wkv_b, w.Dn, out, stream=stream)
+        if evs:
+            evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.fill_(float(i))
+            step(evs[i])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    comb_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    abs_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    up_ms = [e[3].elapsed_time(e[4]) for e in evs]
+    mean_step = sum(step_ms) / K
+    mean_dec = sum(dec_ms) / K
+
+    # end to end: H2D of this step's queries from pinned memory, the four calls, D2H of out
+    h_qn = q_nope.cpu().pin_memory()
+    h_qp = q_pe.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=dt).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for _ in range(3):
+        q_nope.copy_(h_qn, non_blocking=True)
+        q_pe.copy_(h_qp, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    for i in range(K):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        q_nope.copy_(h_qn, non_blocking=True)
+        q_pe.copy_(h_qp, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_mean = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / K
+
+    stats = torch.tensor([mean_step, mean_dec, e2e_mean], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    mean_step, mean_dec, e2e_mean = stats.tolist()
+    if rank != 0:
+        return None
+
+    peaks, psrc = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tflops = peaks["bf16_tflops"]
+    alg = algorithmic(w)
+    dec_gbs = alg["decode_bytes"] / (mean_dec * 1e-3) / 1e9
+    step_gbs = alg["step_bytes"] / (mean_step * 1e-3) / 1e9
+    step_tf = alg["step_flops"] / (mean_step * 1e-3) / 1e12
+    roof_s = max(alg["step_bytes"] / (hbm * 1e9), alg["step_flops"] / (tflops * 1e12))
+    tokens = w.B * w.Q * world
+    value = tokens / (mean_step * 1e-3)
+    pct = lambda xs, q: float(np.percentile(np.asarray(xs), q))
+    res = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(mean_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) inputs, wkv_b N(0,1)/sqrt(512), no trained weights)",
+        "config": dict(workload_desc(w), parallelism=f"dp{world}" if world > 1 else "single GPU",
+                       num_splits=call.num_splits),
+        "roofline": {
+            "kernel": "mla_decode (decode kernel, one launch per step)",
+            "bound": "hbm",
+            "achieved": round(dec_gbs, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(dec_gbs / hbm, 4),
+            "traffic": profiled_traffic(args.workload),
+            "peak_source": f"hbm_gbs of {psrc}",
+            "algorithmic_bytes_per_launch": int(alg["decode_bytes"]),
+        },
+        "step": {
+            "bytes": int(alg["step_bytes"]), "flops": int(alg["step_flops"]),
+            "TB_per_s": round(step_gbs / 1e3, 4), "TFLOP_per_s": round(step_tf, 2),
+            "roofline_us": round(roof_s * 1e6, 2),
+            "roofline_frac": round(roof_s / (mean_step * 1e-3), 4),
+            "roofline_basis": f"max(bytes/{hbm} GB/s, flops/{tflops} TFLOP/s) of {psrc}",
+            "p50_ms": round(pct(step_ms, 50), 5), "p95_ms": round(pct(step_ms, 95), 5),
+            "p99_ms": round(pct(step_ms, 99), 5),
+            "kernel_ms": {"absorb": round(sum(abs_ms) / K, 5), "decode": round(mean_dec, 5),
+                          "combine": round(sum(comb_ms) / K, 5), "up_proj": round(sum(up_ms) / K, 5)},
+        },
+        "e2e": {
+            "value": round(tokens / (e2e_mean * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(e2e_mean, 5),
+            "h2d_bytes_per_step": int(q_nope.numel() * q_nope.element_size() +
+                                      q_pe.numel() * q_pe.element_size()),
+            "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+            "path": "pinned host q_nope/q_pe -> mla_absorb_q -> mla_decode -> mla_combine -> "
+                    "mla_up_proj -> pinned host out, one stream",
+        },
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk.summary(),
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": tflops, "source": psrc},
+    }
+    return res
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def time_oracle(w, budget_s: float = 12.0, min_seqs: int = 1):
+    """Run the fp64 oracle sequence by sequence until ``budget_s`` passes.
+
+    Returns (tokens/s, seconds, sequences, cores). BLAS is held to one thread
+    (einsum's own loops are single-threaded), so cores = 1.
+    """
+    from threadpoolctl import threadpool_limits
+
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from harness import oracle_step
+
+    done, t0 = 0, time.perf_counter()
+    with threadpool_limits(limits=1):
+        while done < w.B and (done < min_seqs or time.perf_counter() - t0 < budget_s):
+            oracle_step(w, batch=[done])
+            done += 1
+    el = time.perf_counter() - t0
+    return done * w.Q / el, el, done, 1
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    w = make_workload(args.workload, 0)
+    per_step = []
+    seqs_done = 0
+    for _ in range(args.warmup + args.steps):
+        tps, el, n, cores = time_oracle(w, budget_s=args.ref_budget)
+        per_step.append(el / (n * w.Q))
+        seqs_done = n
+    sec_per_token = sum(per_step[args.warmup:]) / max(1, args.steps)
+    value = 1.0 / sec_per_token
+    res = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec_per_token * w.B * w.Q * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) inputs, wkv_b N(0,1)/sqrt(512), no trained weights)",
+        "config": dict(workload_desc(w), parallelism="host cores"),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{seqs_done} of {w.B} sequences per step (whole step "
+                                   f"scaled by token count), fp64 NumPy, 1 thread"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dsv3_b64_lk4096")
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--ref-budget", type=float, default=4.0,
+                    help="seconds of oracle work per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if res is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                w = make_workload(args.workload, 0)
+                tps, el, n, cores = time_oracle(w, budget_s=15.0)
+                res["cpu_baseline"] = {"value": round(tps, 3), "unit": "tokens/s", "cores": cores,
+                                       "kind": "oracle",
+                                       "sample": f"{n} of {w.B} sequences of the same workload, "
+                                                 f"fp64 NumPy oracle, {el:.1f} s, 1 thread"}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,18 @@
+// Host-side launchers of libmla's kernels (internal; the public ABI is include/mla.h).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+cudaError_t launch_absorb_simt(const void* q_nope, const void* wkv_b, void* q_lat, int B, int H,
+                               int Q, int Dn, int Vd, int Ckv, bool bf16, cudaStream_t st);
+cudaError_t launch_up_proj_simt(const void* x, const void* wkv_b, void* out, int B, int H, int Q,
+                                int Dn, int Vd, int Ckv, bool bf16, cudaStream_t st);
+size_t decode_simt_smem(int D);
+cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaStream_t st);
+cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
+
+}  // namespace mla

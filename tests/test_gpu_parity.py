@@ -1,0 +1,163 @@
+"""GPU parity: libmla through its C ABI vs the fp64 oracle on the same seeded inputs.
+
+Each ABI call is checked on its own (the oracle stage is fed the GPU's
+previous output) and end to end. Small cases span several 64-token tiles and
+a ragged tail; full-size workloads are checked on sampled sequences.
+"""
+import numpy as np
+import pytest
+import torch
+
+from latent_kv_decode_b200 import workloads as wl
+from oracle import mla as omla
+
+from harness import (TOL_BF16, TOL_F32, REL_L2_BF16, assert_close, dev, fp4_entries, gpu_shared_latent,
+                     gpu_step, oracle_shared_latent, oracle_step, upload)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_step(w, g, batch=None, tol=None, rel=None):
+    tol = tol or (TOL_F32 if w.dtype == "f32" else TOL_BF16)
+    rel = rel if rel is not None else (None if w.dtype == "f32" else REL_L2_BF16)
+    sel = slice(None) if batch is None else np.asarray(batch)
+    ref = oracle_step(w, batch)
+    assert_close(g["q_lat"][sel], ref["q_lat"], tol, "q_lat", rel)
+    # decode on the GPU's own q_lat, up-projection on the GPU's own x
+    ref_x = oracle_step(w, batch, q_lat=g["q_lat"][sel])
+    assert_close(g["x"][sel], ref_x["x"], tol, "x", rel)
+    assert_close(g["lse"][sel], ref_x["lse"], tol, "lse")
+    ref_o = oracle_step(w, batch, x=g["x"][sel])
+    assert_close(g["out"][sel], ref_o["out"], tol, "out(up_proj)", rel)
+    assert_close(g["out"][sel], ref["out"], tol, "out(end to end)", rel)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_demo_fp32(splits):
+    w = wl.demo_fp32()
+    g = gpu_step(w, upload(w), num_splits=splits)
+    assert g["out"].shape == (2, 8, 1, 128)
+    _check_step(w, g)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5, 0])
+@pytest.mark.parametrize("combined", [False, True])
+def test_dsv3_small_ragged_tail(splits, combined):
+    w = wl.dsv3(B=3, Lk=333, seed=11)
+    _check_step(w, gpu_step(w, upload(w, combined), num_splits=splits))
+
+
+def test_fp32_dsv3_dims():
+    w = wl.make_mla(2, 16, 1, 128, 64, 128, 512, 150, dtype="f32", seed=12)
+    _check_step(w, gpu_step(w, upload(w), num_splits=2))
+
+
+@pytest.mark.parametrize("splits", [1, 4])
+def test_seq_lens_mask_and_causal_q2(splits):
+    mask = np.ones(300, np.uint8)
+    mask[[0, 17, 64, 65, 299]] = 0
+    w = wl.make_mla(4, 128, 2, 128, 64, 128, 512, 300, dtype="bf16", seed=13,
+                    seq_lens=[300, 1, 65, 129], causal=True, causal_mask=mask)
+    _check_step(w, gpu_step(w, upload(w), num_splits=splits))
+
+
+@pytest.mark.parametrize("combined", [False, True])
+def test_paged_ragged_q2(combined):
+    w = wl.make_mla(5, 128, 2, 128, 64, 128, 512, 0, dtype="bf16", seed=14, lk_range=(2, 700),
+                    paged=True, causal=True)
+    _check_step(w, gpu_step(w, upload(w, combined), num_splits=0))
+
+
+def test_more_splits_than_tiles_leaves_empty_splits():
+    w = wl.dsv3(B=2, Lk=100, seed=15)
+    _check_step(w, gpu_step(w, upload(w), num_splits=7))
+
+
+def test_single_token_cache():
+    w = wl.dsv3(B=2, Lk=1, seed=16)
+    _check_step(w, gpu_step(w, upload(w), num_splits=1))
+
+
+def test_fully_masked_rows_are_zero():
+    mask = np.zeros(70, np.uint8)
+    w = wl.make_mla(2, 8, 1, 64, 32, 128, 512, 70, dtype="f32", seed=17, causal_mask=mask)
+    g = gpu_step(w, upload(w), num_splits=2)
+    assert np.all(g["x"] == 0) and np.all(g["out"] == 0) and np.all(np.isneginf(g["lse"]))
+
+
+def test_bad_block_table_entry_sets_flag_and_skips_page():
+    w = wl.make_mla(2, 8, 1, 64, 32, 128, 512, 0, dtype="f32", seed=18, seq_lens=[200, 130],
+                    paged=True)
+    d = upload(w)
+    bt = w.block_table.copy()
+    bt[0, 1] = 10_000                      # page 1 of sequence 0 is out of range
+    d["block_table"] = dev(bt)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = gpu_step(w, d, num_splits=2, err_flag=flag)
+    assert int(flag.item()) & 1
+    # expected: the same decode with tokens 64..127 of sequence 0 invisible
+    mask_w = wl.make_mla(2, 8, 1, 64, 32, 128, 512, 0, dtype="f32", seed=18, seq_lens=[200, 130],
+                         paged=True)
+    kv = omla.gather_paged(mask_w.kv_pool, mask_w.block_table, mask_w.lens(), 64)
+    pe = omla.gather_paged(mask_w.pe_pool, mask_w.block_table, mask_w.lens(), 64)
+    vis = omla.visibility(2, 1, kv.shape[1], mask_w.seq_lens)
+    vis[0, :, 64:128] = False
+    x, _, _ = omla.latent_attention(g["q_lat"], w.q_pe, kv, pe, w.softmax_scale, vis)
+    assert_close(g["x"], x, TOL_F32, "x with skipped page")
+
+
+# --- shared-latent FP4 variant ----------------------------------------------
+
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_shared_latent_fp4_small(splits):
+    w = wl.make_shared_latent(3, 64, 1, 333, seed=21, seq_lens=[333, 64, 200])
+    ent = fp4_entries(w)
+    g = gpu_shared_latent(w, ent, num_splits=splits)
+    ref = oracle_shared_latent(w, ent)
+    assert_close(g["x"], ref["x"], TOL_BF16, "x", REL_L2_BF16)
+    assert_close(g["lse"], ref["lse"], TOL_BF16, "lse")
+
+
+def test_shared_latent_fp4_paged():
+    w = wl.make_shared_latent(3, 64, 1, 260, seed=22, seq_lens=[260, 65, 3], paged=True)
+    ent = fp4_entries(w)
+    g = gpu_shared_latent(w, ent, num_splits=2, paged=True)
+    ref = oracle_shared_latent(w, ent)
+    assert_close(g["x"], ref["x"], TOL_BF16, "x", REL_L2_BF16)
+
+
+# --- full-size workloads, sampled sequences ----------------------------------
+
+@pytest.mark.slow
+def test_full_dsv3_b64_lk4096():
+    w = wl.dsv3()
+    g = gpu_step(w, upload(w))
+    _check_step(w, g, batch=[0, 31, 63])
+
+
+@pytest.mark.slow
+def test_full_longctx_b4_lk131072():
+    w = wl.longctx()
+    g = gpu_step(w, upload(w))
+    assert g["splits"] > 1
+    _check_step(w, g, batch=[0, 3])
+
+
+@pytest.mark.slow
+def test_full_ragged_paged_b128_q2():
+    w = wl.ragged_paged()
+    g = gpu_step(w, upload(w))
+    L = w.lens()
+    batch = [int(np.argmin(L)), int(np.argmax(L)), 5]
+    _check_step(w, g, batch=batch)
+
+
+@pytest.mark.slow
+def test_full_v41_fp4_sink_h64():
+    w = wl.v41_shared_latent()
+    ent = fp4_entries(w)
+    g = gpu_shared_latent(w, ent)
+    batch = [0, 17, 31]
+    ref = oracle_shared_latent(w, ent, batch)
+    assert_close(g["x"][batch], ref["x"], TOL_BF16, "x", REL_L2_BF16)
+    assert_close(g["lse"][batch], ref["lse"], TOL_BF16, "lse")
