@@ -58,8 +58,9 @@ def load_peaks():
 
 def make_workload(name: str, rank: int):
     from latent_kv_decode_b200 import workloads as wl
-    if name == "dsv3_b64_lk4096":
-        return wl.dsv3(seed=1 + 1000 * rank)
+    m = re.fullmatch(r"dsv3_b(\d+)_lk(\d+)", name)
+    if m:
+        return wl.dsv3(B=int(m.group(1)), Lk=int(m.group(2)), seed=1 + 1000 * rank)
     if name == "longctx_b4_lk131072":
         return wl.longctx(seed=3 + 1000 * rank)
     if name == "ragged_paged_b128_q2":
@@ -80,9 +81,9 @@ def workload_desc(w) -> dict:
 def algorithmic(w):
     """Algorithmic bytes / flops of one step and of the decode launch.
 
-    Decode: every visible cache row once (Ckv+Dr elements), q_lat and q_pe
-    read once, x written once. Step: plus W_UK and W_UV read once, q_nope read,
-    q_lat written and read, x read, out written. Flops: 2*H*Q*(Ckv+Dr) per
+    Decode launch: every cache row once (Ckv+Dr elements), q_lat and q_pe
+    read once, x written once. Step: cache rows, wkv_b (W_UK and W_UV), q_nope,
+    q_pe and out, each once (340,787,200 B for B=64, Lk=4096). Flops: 2*H*Q*(Ckv+Dr) per
     visible token for the scores and 2*H*Q*Ckv for the aggregation, plus the
     two projections 2*B*Q*H*Ckv*(Dn+Vd).
     """
@@ -96,11 +97,13 @@ def algorithmic(w):
     HQ = w.H * w.Q
     dec_bytes = rows_read * (w.Ckv + w.Dr) * es + w.B * HQ * (w.Ckv + w.Dr) * es + w.B * HQ * w.Ckv * es
     dec_flops = vis_rows * w.Q * w.H * 2 * ((w.Ckv + w.Dr) + w.Ckv)
-    proj_bytes = (w.H * (w.Dn + w.Vd) * w.Ckv * es + w.B * HQ * w.Dn * es + w.B * HQ * w.Ckv * es
-                  + w.B * HQ * w.Ckv * es + w.B * HQ * w.Vd * es)
+    # the step's unavoidable traffic: cache rows, wkv_b, the queries and the output
+    # (q_lat and x are intermediates a fused step would not write)
+    step_bytes = (rows_read * (w.Ckv + w.Dr) * es + w.H * (w.Dn + w.Vd) * w.Ckv * es
+                  + w.B * HQ * (w.Dn + w.Dr) * es + w.B * HQ * w.Vd * es)
     proj_flops = 2 * w.B * HQ * w.Ckv * (w.Dn + w.Vd)
     return dict(decode_bytes=dec_bytes, decode_flops=dec_flops,
-                step_bytes=dec_bytes + proj_bytes, step_flops=dec_flops + proj_flops)
+                step_bytes=step_bytes, step_flops=dec_flops + proj_flops)
 
 
 class ClockSampler:
