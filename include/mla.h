@@ -197,6 +197,36 @@ mla_status_t mla_decode(const mla_decode_args* a, void* workspace, size_t worksp
 mla_status_t mla_combine(const mla_decode_args* a, const void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/*
+ * mla_decode_static_scratch - mla_decode followed by mla_combine, for callers
+ * that may not allocate device memory. The paper has no counterpart: this is
+ * a deployment variant of the two calls above.
+ *
+ * Some callers cannot call cudaMalloc or take memory from an allocator: a
+ * serving engine that reserved nearly all of HBM for its KV cache at start-up
+ * (an allocation at decode time would fail), or a plugin hook of a host
+ * runtime that forbids allocation inside the hook. This entry point needs no
+ * workspace argument: the split-KV partials go to one array of
+ * MLA_STATIC_SCRATCH_BYTES bytes of device memory that the library owns,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   - Takes the same arguments as mla_decode and writes a->x and a->lse; they
+ *     are final when the work it enqueued on `stream` completes.
+ *   - Returns MLA_ERR_WORKSPACE, enqueuing nothing, when the resolved split
+ *     count needs more than MLA_STATIC_SCRATCH_BYTES (see
+ *     mla_decode_workspace_size); one split needs no scratch at all.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array, whatever the stream. Calls whose GPU
+ *     work overlaps in time race on it and give wrong results: serialise them
+ *     (one stream, or events). The array keeps the last call's contents;
+ *     nothing in it needs to start at zero, because mla_decode writes every
+ *     partial that mla_combine reads in the same call.
+ *   - Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MLA_STATIC_SCRATCH_BYTES (32u << 20)
+mla_status_t mla_decode_static_scratch(const mla_decode_args* a, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -232,3 +234,53 @@ mla_status_t mla_combine(const mla_decode_args* a, const void* workspace, size_t
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation: the split-KV partials live in a
+// library-owned array in device memory instead of a caller workspace.
+// ---------------------------------------------------------------------------
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[MLA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device. Host code only
+// sees a host-side stand-in for the array, so the address is looked up once
+// per device, with that device current, and cached.
+mla_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status_t mla_decode_static_scratch(const mla_decode_args* a, void* stream) {
+  mla_status_t s = validate_decode(a);
+  if (s != MLA_OK) return s;
+  const size_t need = ws_bytes(a, resolve_splits(a));
+  if (need > (size_t)MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    s = static_scratch_address(&ws);
+    if (s != MLA_OK) return s;
+  }
+  s = mla_decode(a, ws, need, stream);
+  if (s != MLA_OK) return s;
+  return mla_combine(a, ws, need, stream);
+}

@@ -50,6 +50,7 @@ _SIGS = {
     "mla_decode_workspace_size": (_c.c_size_t, [_c.c_void_p]),
     "mla_decode": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "mla_combine": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "mla_decode_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
 }
 
 
@@ -264,6 +265,20 @@ def mla_combine(call: DecodeCall, stream=None) -> DecodeCall:
     ws = call.workspace
     _check(lib().mla_combine(ctypes.byref(call.args), _ptr(ws) if need else None, need,
                              _stream(stream)), "mla_combine")
+    return call
+
+
+def mla_decode_static_scratch(call: DecodeCall, stream=None) -> DecodeCall:
+    """Decode and combine with the library's own scratch array: no workspace, no allocation.
+
+    For callers that may not allocate device memory at decode time. The
+    call's ``x``/``lse`` are final once the enqueued work completes. Raises
+    when the split count needs more than MLA_STATIC_SCRATCH_BYTES (32 MiB).
+    All such calls share one array per device: keep them from overlapping
+    on the GPU.
+    """
+    _check(lib().mla_decode_static_scratch(ctypes.byref(call.args), _stream(stream)),
+           "mla_decode_static_scratch")
     return call
 
 
