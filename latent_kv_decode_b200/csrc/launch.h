@@ -15,4 +15,9 @@ size_t decode_simt_smem(int D);
 cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaStream_t st);
 cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
 
+// tensor-core (tcgen05, 2-CTA cluster) decode for bf16, Ckv=512, Dr=64, H*Q % 128 == 0
+bool sm100_decode_supported(const mla_decode_args* a);
+int sm100_auto_splits(const mla_decode_args* a, int sms);
+cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a, cudaStream_t st);
+
 }  // namespace mla

@@ -57,6 +57,9 @@ def upload(w: wl.Workload, combined: bool = False) -> dict:
 def gpu_step(w: wl.Workload, d: dict, num_splits: int = 0, err_flag=None):
     """absorb -> decode -> combine -> up_proj through the C ABI; returns numpy dict."""
     from latent_kv_decode_b200 import ops
+    own_flag = err_flag is None
+    if own_flag:
+        err_flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     q_lat = ops.mla_absorb_q(d["q_nope"], d["wkv_b"])
     call = ops.mla_decode(q_lat, d["q_pe"], d["kv"], d["pe"], w.softmax_scale,
                           seq_lens=d["seq_lens"], block_table=d["block_table"],
@@ -66,6 +69,8 @@ def gpu_step(w: wl.Workload, d: dict, num_splits: int = 0, err_flag=None):
     ops.mla_combine(call)
     out = ops.mla_up_proj(call.x, d["wkv_b"], w.Dn)
     torch.cuda.synchronize()
+    if own_flag:
+        assert int(err_flag.item()) == 0, f"kernel reported device error bits {int(err_flag.item())}"
     f = lambda t: t.float().cpu().numpy().astype(np.float64)
     return dict(q_lat=f(q_lat), x=f(call.x), lse=f(call.lse), out=f(out), splits=call.num_splits)
 
@@ -149,13 +154,15 @@ def gpu_shared_latent(w: wl.Workload, entries: np.ndarray, num_splits: int = 0, 
     else:
         kv, bt = dev(entries), None
     sinks = dev(w.sinks.astype(np.float32)) if w.sinks is not None else None
+    err_flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     call = ops.mla_decode(q, None, kv, None, w.softmax_scale,
                           seq_lens=dev(w.seq_lens) if w.seq_lens is not None else None,
                           block_table=bt, page_size=w.page_size, causal=w.causal, sinks=sinks,
                           rope_tail=w.rope_tail, rope_theta=w.rope_theta, num_splits=num_splits,
-                          Lk=w.Lk if bt is None else None)
+                          Lk=w.Lk if bt is None else None, err_flag=err_flag)
     ops.mla_combine(call)
     torch.cuda.synchronize()
+    assert int(err_flag.item()) == 0, f"kernel reported device error bits {int(err_flag.item())}"
     return dict(x=call.x.float().cpu().numpy().astype(np.float64),
                 lse=call.lse.cpu().numpy().astype(np.float64), splits=call.num_splits)
 
