@@ -7,23 +7,27 @@
 // (tcgen05 cta_group::2, M = 128), so each SM computes its own 64 rows at the
 // full datapath width. Per 128-token tile of the cache:
 //
-//   S  = Q . K^T   9 chunks of 64 dims (8 latent + 1 rope). CTA r supplies
-//                  tokens [64r, 64r+64) of each chunk (the N half of B).
+//   S  = Q . K^T   over the 576 dims in 64-dim chunks (8 latent + 1 rope).
+//                  CTA r supplies tokens [64r, 64r+64) of the tile (the N half
+//                  of B), loaded as 4 stages of 2 latent chunks + 1 rope stage.
 //   softmax        online, base 2, lazy rescale (the running max only moves
 //                  when a score exceeds it by more than 2^8).
-//   O += P . V     4 chunks of 32 tokens x 2 halves of 256 latent columns.
-//                  CTA r supplies latent columns [128r, 128r+128) of each half.
+//   O += P . V     2 halves of 256 latent columns x 2 halves of 64 tokens.
+//                  CTA r supplies latent columns [128r, 128r+128) of each half
+//                  for all 128 tokens.
 //
 // The latent rows are therefore read twice per tile (once as K, once as V,
-// cut differently between the pair); the second read is an L2 hit, so HBM
-// sees each cache row once. Scores and the output accumulator live in TMEM
-// (S double-buffered: 2 x 64 columns; O: 2 x 128 columns); tiles arrive by
-// TMA into a 12-stage ring of 8 KB chunks per CTA.
+// cut differently between the pair); the K producer prefetches whole row
+// ranges into L2 three tiles ahead, so HBM sees each cache row once and both
+// shared-memory loads are L2 hits. Every TMA request moves 64 rows x 2 chunks
+// (16 KB) through a 4-D view of the cache whose box lands already in the
+// 128-byte-swizzled layout the MMAs read. Scores and the output accumulator
+// live in TMEM (S double-buffered: 2 x 64 columns; O: 2 x 128 columns).
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer (even CTA
-// only) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane = 32*(warp%4)
-// + lane). Every wait is bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and the
-// kernel unwinds.
+// Warp roles (224 threads): warp 0 K producer (+ Q), warp 1 MMA issuer (even
+// CTA only) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane =
+// 32*(warp%4) + lane), warp 6 V producer. Every wait is bounded; a timeout sets
+// MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -36,22 +40,28 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kTileT = 128;                 // tokens per tile (both CTAs)
-constexpr int kStages = 12;
-constexpr int kChunk = 8192;                // bytes per CTA per stage
+constexpr int kKStages = 5;                 // ring of K stages (16 KB: 2 latent chunks, or rope): a tile
+constexpr int kVStages = 3;                 // ring of V stages (16 KB; a tile uses 4)
+constexpr int kStage = 16384;               // bytes per CTA per stage
+constexpr int kKUses = 5;                   // K stage uses per tile: 4 latent pairs + rope
+constexpr int kPrefetchTiles = 0;           // L2 prefetch distance of the K producer (off: measured no gain)
 constexpr int kQBlocks = 9;                 // 64-dim blocks of the 576-wide query row
 constexpr int kQBytes = kQBlocks * 8192;    // 64 rows x 128 B per block
-constexpr int kPBuf = 16384;                // 64 rows x 128 tokens bf16 (2 blocks)
+constexpr int kPBuf = 16384;                // P: 64 rows x 128 tokens bf16 (2 blocks), one buffer
 
 constexpr int kOffQ = 0;
-constexpr int kOffStage = kOffQ + kQBytes;
-constexpr int kOffP = kOffStage + kStages * kChunk;
-constexpr int kOffBar = kOffP + 2 * kPBuf;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKStages * kStage;
+constexpr int kOffP = kOffV + kVStages * kStage;
+constexpr int kOffBar = kOffP + kPBuf;
 enum : int {
-  B_FULL = 0,
-  B_EMPTY = B_FULL + kStages,
-  B_QFULL = B_EMPTY + kStages,
+  B_KFULL = 0,
+  B_KEMPTY = B_KFULL + kKStages,
+  B_VFULL = B_KEMPTY + kKStages,
+  B_VEMPTY = B_VFULL + kVStages,
+  B_QFULL = B_VEMPTY + kVStages,
   B_SFULL = B_QFULL + 1,
   B_SFREE = B_SFULL + 2,
   B_PFULL = B_SFREE + 2,
@@ -75,12 +85,23 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct alignas(64) Sm100Params {
   CUtensorMap tm_q;    // q_lat  (B*HQ, 512), box 64 x 64
   CUtensorMap tm_qpe;  // q_pe   (B*HQ, 64),  box 64 x 64
-  CUtensorMap tm_k;    // latent cache, box 64 dims x 64 tokens
-  CUtensorMap tm_v;    // latent cache, box 64 dims x 32 tokens
-  CUtensorMap tm_pe;   // rope cache,   box 64 dims x 64 tokens
+  CUtensorMap tm_k;    // latent cache as (64 dims, rows, 8 chunks, seq|page): box 64 rows x 2 chunks
+  CUtensorMap tm_pe;   // rope cache (64 dims, rows, seq|page): box 64 rows
   DecodeParams p;
   int paged;
 };
+
+// 2^x on the SFU; subnormal results flush to zero (probabilities below
+// 2^-126 of the row maximum are irrelevant at bf16 precision).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 __device__ __forceinline__ bool bar_or(int id, int count, bool pred) {
   uint32_t out;
@@ -132,15 +153,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(B_FULL + s), 1);
-      mbar_init(bar(B_EMPTY + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
     }
     mbar_init(bar(B_QFULL), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_SFREE + i), 8);
-      mbar_init(bar(B_PFULL + i), 8);
+      mbar_init(bar(B_SFREE + i), 2);   // one arrival per CTA
+      mbar_init(bar(B_PFULL + i), 2);   // one arrival per CTA
       mbar_init(bar(B_PVDONE + i), 1);
     }
     *abort_flag = 0;
@@ -159,138 +184,186 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     *abort_flag = 1;
     flag_error(p, MLA_DEVICE_ERR_TIMEOUT);
   };
+  // let copies already issued land before this CTA's shared memory goes away
+  auto settle = []() {
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 50000ull) {
+    }
+  };
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ K producer
+    // Q once, then for every tile the 9 K chunks (this CTA's 64 tokens x 64 dims).
     if (lane == 0) {
       tma_prefetch_desc(&P.tm_q);
+      tma_prefetch_desc(&P.tm_qpe);
       tma_prefetch_desc(&P.tm_k);
-      tma_prefetch_desc(&P.tm_v);
       tma_prefetch_desc(&P.tm_pe);
       const int qrow = b * p.HQ + rb * 128 + (int)rank * 64;
       const uint32_t qbar = map_to_rank(bar(B_QFULL), 0);
       if (rank == 0) mbar_arrive_expect_tx(bar(B_QFULL), 2 * kQBytes);
       for (int c = 0; c < 8; ++c) tma_load_2d_2sm(sb0 + kOffQ + c * 8192, &P.tm_q, qbar, 64 * c, qrow);
       tma_load_2d_2sm(sb0 + kOffQ + 8 * 8192, &P.tm_qpe, qbar, 0, qrow);
-
+      // L2 prefetch of this CTA's 64 cache rows of a tile (latent and rope rows
+      // as whole contiguous ranges), kPrefetchTiles ahead of the shared-memory loads
+      auto prefetch_tile = [&](int jt) {
+        const int t = t_begin + jt * kTileT + (int)rank * 64;
+        if (jt >= ntiles || t >= len) return;
+        const int rows = min(64, len - t);
+        const char* kvb = reinterpret_cast<const char*>(p.kv);
+        const char* peb = reinterpret_cast<const char*>(p.pe);
+        if (P.paged) {
+          const int64_t row0 = (int64_t)page_of(p, b, t, len) * 64;
+          kvb += row0 * p.kv_row * 2;
+          peb += row0 * p.pe_row * 2;
+        } else {
+          kvb += ((int64_t)b * p.kv_batch + (int64_t)t * p.kv_row) * 2;
+          peb += ((int64_t)b * p.pe_batch + (int64_t)t * p.pe_row) * 2;
+        }
+        // the range ends at the last row's own data (strided rows may share a buffer)
+        prefetch_l2_bulk(kvb, (uint32_t)(((int64_t)(rows - 1) * p.kv_row + p.Ckv) * 2));
+        prefetch_l2_bulk(peb, (uint32_t)(((int64_t)(rows - 1) * p.pe_row + p.Dr) * 2));
+      };
+      for (int jt = 0; jt < kPrefetchTiles; ++jt) prefetch_tile(jt);
       uint32_t it = 0;
       bool ok = true;
-      // Claim the next ring stage: wait until the MMAs released it, arm its
-      // full barrier (in the even CTA) for both CTAs' bytes.
-      auto acquire = [&](uint32_t& dst, uint32_t& fbar) -> bool {
-        const uint32_t s = it % kStages, round = it / kStages;
-        if (round > 0 && !mbar_wait_cluster(bar(B_EMPTY + s), (round - 1) & 1)) return false;
-        if (rank == 0) mbar_arrive_expect_tx(bar(B_FULL + s), 2 * kChunk);
-        dst = sb0 + kOffStage + s * kChunk;
-        fbar = map_to_rank(bar(B_FULL + s), 0);
-        ++it;
-        return true;
-      };
-      for (int j = 0; j <= ntiles && ok; ++j) {
-        if (j < ntiles) {
-          // K chunks of tile j: this CTA's 64 tokens, 9 blocks of 64 dims
-          const int t = t_begin + j * kTileT + (int)rank * 64;
-          int y = t, zc = b;
-          if (P.paged) {
-            zc = page_of(p, b, t, len);
-            y = 0;
-          }
-          for (int c = 0; c < kQBlocks && ok; ++c) {
-            uint32_t dst, fb;
-            if (!acquire(dst, fb)) { ok = false; break; }
-            if (c < 8)
-              tma_load_3d_2sm(dst, &P.tm_k, fb, 64 * c, y, zc);
-            else
-              tma_load_3d_2sm(dst, &P.tm_pe, fb, 0, y, zc);
-          }
+      for (int j = 0; j < ntiles && ok; ++j) {
+        if (kPrefetchTiles > 0) prefetch_tile(j + kPrefetchTiles);
+        const int t = t_begin + j * kTileT + (int)rank * 64;
+        int y = t, zc = b;
+        if (P.paged) {
+          zc = page_of(p, b, t, len);
+          y = 0;
         }
-        if (j >= 1 && ok) {
-          // V chunks of tile j-1: 32 tokens x this CTA's 128 columns of each 256-half
-          const int tj = t_begin + (j - 1) * kTileT;
-          for (int kc = 0; kc < 4 && ok; ++kc) {
-            const int t = tj + 32 * kc;
-            int y = t, zc = b;
-            if (P.paged) {
-              zc = page_of(p, b, t, len);
-              y = t & 63;
-            }
-            for (int n = 0; n < 2; ++n) {
-              uint32_t dst, fb;
-              if (!acquire(dst, fb)) { ok = false; break; }
-              const int x0 = 256 * n + 128 * (int)rank;
-              tma_load_3d_2sm(dst, &P.tm_v, fb, x0, y, zc);
-              tma_load_3d_2sm(dst + 4096, &P.tm_v, fb, x0 + 64, y, zc);
-            }
+        for (int u = 0; u < kKUses; ++u, ++it) {
+          const uint32_t s = it % kKStages, round = it / kKStages;
+          if (round > 0 && !mbar_wait_cluster(bar(B_KEMPTY + s), (round - 1) & 1)) { ok = false; break; }
+          const uint32_t dst = sb0 + kOffK + s * kStage, fb = map_to_rank(bar(B_KFULL + s), 0);
+          if (u < 4) {
+            if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * kStage);
+            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 2 * u, zc);
+          } else {
+            if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * 8192);
+            tma_load_3d_2sm(dst, &P.tm_pe, fb, 0, y, zc);
           }
         }
         if (*abort_flag) ok = false;
       }
       if (!ok) {
         fail();
-        // let copies already issued land before this CTA's shared memory goes away
-        const uint64_t t0 = global_ns();
-        while (global_ns() - t0 < 50000ull) {
+        settle();
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ V producer
+    // For tile j, after QK(j) has completed (these rows sit in L2): for each
+    // 256-column half and each 64-token half, this CTA's 128 latent columns.
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        if (!mbar_wait_cluster(bar(B_SFULL + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
+        const int tj = t_begin + j * kTileT;
+        for (int n = 0; n < 2 && ok; ++n) {
+          for (int th = 0; th < 2; ++th, ++it) {
+            const int t = tj + 64 * th;
+            int y = t, zc = b;
+            if (P.paged) {
+              zc = page_of(p, b, t, len);
+              y = 0;
+            }
+            const uint32_t s = it % kVStages, round = it / kVStages;
+            if (round > 0 && !mbar_wait_cluster(bar(B_VEMPTY + s), (round - 1) & 1)) { ok = false; break; }
+            if (rank == 0) mbar_arrive_expect_tx(bar(B_VFULL + s), 2 * kStage);
+            const uint32_t dst = sb0 + kOffV + s * kStage, fb = map_to_rank(bar(B_VFULL + s), 0);
+            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 4 * n + 2 * (int)rank, zc);
+          }
         }
+        if (*abort_flag) ok = false;
+      }
+      if (!ok) {
+        fail();
+        settle();
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
+    // Two independent streams, polled: QK(j) (needs S(j-2) released and K
+    // stages) and PV(j) (needs P(j) and V stages). Neither waits on the other,
+    // so a V stage in flight never stalls the K ring and vice versa.
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
       bool ok = mbar_wait_cluster(bar(B_QFULL), 0);
-      uint32_t it = 0;
-      for (int j = 0; j <= ntiles && ok; ++j) {
-        if (j < ntiles) {
-          const int sbuf = j & 1;
-          if (j >= 2 && !mbar_wait_cluster(bar(B_SFREE + sbuf), ((j - 2) >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + kColS + 64u * sbuf;
-          for (int c = 0; c < kQBlocks; ++c) {
-            const uint32_t s = it % kStages;
-            if (!mbar_wait_cluster(bar(B_FULL + s), (it / kStages) & 1)) { ok = false; break; }
+      uint32_t kit = 0, vit = 0;
+      int qj = 0, qu = 0;   // next QK: tile, stage use (4 latent pairs + rope)
+      int pj = 0, pu = 0;   // next PV: tile, stage use (n * 2 + token half)
+      uint64_t t_idle = global_ns();
+      uint32_t idle = 0;
+      while (ok && pj < ntiles) {
+        bool prog = false;
+        if (qj < ntiles) {
+          const int sbuf = qj & 1;
+          const bool sfree = qu > 0 || qj < 2 || mbar_poll_cluster(bar(B_SFREE + sbuf), ((qj - 2) >> 1) & 1);
+          const uint32_t s = kit % kKStages;
+          if (sfree && mbar_poll_cluster(bar(B_KFULL + s), (kit / kKStages) & 1)) {
             tc_fence_after();
-            const uint32_t qa = sb0 + kOffQ + c * 8192, kb = sb0 + kOffStage + s * kChunk;
+            const uint32_t d = tmem + kColS + 64u * sbuf;
+            const uint32_t kb = sb0 + kOffK + s * kStage;
+            const int nch = (qu < 4) ? 2 : 1;
+            for (int cc = 0; cc < nch; ++cc) {
+              const int c = (qu < 4) ? 2 * qu + cc : 8;   // 64-dim block of Q
+              const uint32_t qa = sb0 + kOffQ + c * 8192, ka = kb + cc * 8192;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                mma_bf16_ss_2sm(d, smem_desc(qa + 32 * k, 16, 1024, kSwizzle128B),
+                                smem_desc(ka + 32 * k, 16, 1024, kSwizzle128B), idesc_qk,
+                                (qu | cc | k) != 0);
+              }
+            }
+            mma_commit_2sm_mc(bar(B_KEMPTY + s), 3);
+            ++kit;
+            if (++qu == kKUses) {
+              mma_commit_2sm_mc(bar(B_SFULL + sbuf), 3);
+              qu = 0;
+              ++qj;
+            }
+            prog = true;
+          }
+        }
+        if (pj < qj) {
+          const bool pready = pu > 0 || mbar_poll_cluster(bar(B_PFULL + (pj & 1)), (pj >> 1) & 1);
+          const uint32_t s = vit % kVStages;
+          if (pready && mbar_poll_cluster(bar(B_VFULL + s), (vit / kVStages) & 1)) {
+            tc_fence_after();
+            const int n = pu >> 1, th = pu & 1;
+            const uint32_t vb = sb0 + kOffV + s * kStage;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              mma_bf16_ss_2sm(d, smem_desc(qa + 32 * k, 16, 1024, kSwizzle128B),
-                              smem_desc(kb + 32 * k, 16, 1024, kSwizzle128B), idesc_qk,
-                              (c | k) != 0);
+              // P: K-block th (64 tokens), 16 tokens per step; V: 2 blocks of 64 columns
+              const uint32_t a_addr = sb0 + kOffP + th * 8192 + 32 * k;
+              mma_bf16_ss_2sm(tmem + kColO + 128u * n, smem_desc(a_addr, 16, 1024, kSwizzle128B),
+                              smem_desc(vb + 2048 * k, 8192, 1024, kSwizzle128B), idesc_pv,
+                              (pj > 0 || th > 0 || k > 0) ? 1u : 0u);
             }
-            mma_commit_2sm_mc(bar(B_EMPTY + s), 3);
-            ++it;
-          }
-          if (!ok) break;
-          mma_commit_2sm_mc(bar(B_SFULL + sbuf), 3);
-        }
-        if (j >= 1) {
-          const int jj = j - 1, sbuf = jj & 1;
-          if (!mbar_wait_cluster(bar(B_PFULL + sbuf), (jj >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t pa = sb0 + kOffP + sbuf * kPBuf;
-          for (int kc = 0; kc < 4 && ok; ++kc) {
-            for (int n = 0; n < 2; ++n) {
-              const uint32_t s = it % kStages;
-              if (!mbar_wait_cluster(bar(B_FULL + s), (it / kStages) & 1)) { ok = false; break; }
-              tc_fence_after();
-              const uint32_t vb = sb0 + kOffStage + s * kChunk;
-#pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                const uint32_t a_addr = pa + (kc >> 1) * 8192 + (kc & 1) * 64 + 32 * k;
-                mma_bf16_ss_2sm(tmem + kColO + 128u * n,
-                                smem_desc(a_addr, 16, 1024, kSwizzle128B),
-                                smem_desc(vb + 2048 * k, 4096, 1024, kSwizzle128B), idesc_pv,
-                                (jj > 0 || kc > 0 || k > 0) ? 1u : 0u);
-              }
-              mma_commit_2sm_mc(bar(B_EMPTY + s), 3);
-              ++it;
+            mma_commit_2sm_mc(bar(B_VEMPTY + s), 3);
+            ++vit;
+            if (++pu == 4) {
+              mma_commit_2sm_mc(bar(B_PVDONE + (pj & 1)), 3);
+              pu = 0;
+              ++pj;
             }
+            prog = true;
           }
-          if (!ok) break;
-          mma_commit_2sm_mc(bar(B_PVDONE + sbuf), 3);
         }
-        if (*abort_flag) ok = false;
+        if (prog) {
+          idle = 0;
+        } else if ((++idle & 255u) == 0) {
+          if (idle == 256u) t_idle = global_ns();
+          else if (global_ns() - t_idle > 1000000000ull || *abort_flag) ok = false;
+        }
       }
       if (!ok) fail();
     }
@@ -308,6 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     float* xsum = xmax + 256;
     float m_run = -INFINITY, l_part = 0.f;
     bool ab = false;
+    // loop-invariant parameters, read once into registers
+    const float sl2 = p.scale_log2;
+    const uint8_t* mask = p.mask;
+    const bool causal = p.causal != 0;
+    const int causal_last = len - p.Q + q;   // last visible token of a causal row
+    const bool paged = p.block_table != nullptr;
+    const bool leader_thread = (L == 0);     // arrives for this CTA on the even CTA's barriers
 
     for (int j = 0; j < ntiles; ++j) {
       const int sbuf = j & 1;
@@ -324,24 +404,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(v[c][i]);
-        tc_fence_before();
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(bar(B_SFREE + sbuf), 0));
+      tc_fence_before();
 
-      // scale to log2 units and mask: this thread holds tokens [tb, tb + 64)
+      // scale to log2 units and mask: this thread holds tokens [tb, tb + 64);
+      // tokens [tb, tb + lim) pass the range / causal / page tests
       const int tb = t_begin + j * kTileT + 64 * half;
-      const bool pg_ok = page_ok(p, b, tb < len ? tb : 0);
+      int lim = t_end - tb;
+      if (causal) lim = min(lim, causal_last - tb + 1);
+      if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;
+      if (ab) lim = 0;
       float mx = -INFINITY;
+      if (mask == nullptr) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int t = tb + c;
-        const bool vis = !ab && pg_ok && t < t_end && visible(p, len, q, t);
-        s[c] = vis ? s[c] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; ++c) {
+          s[c] = (c < lim) ? s[c] * sl2 : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const bool vis = c < lim && mask[tb + c] != 0;
+          s[c] = vis ? s[c] * sl2 : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
       }
       xmax[sbuf * 128 + L] = mx;
-      if (bar_or(1, 128, ab)) {
+      // all four warps have read S(j) by now: release the buffer to the MMA
+      const bool stop = bar_or(1, 128, ab);
+      if (leader_thread) mbar_arrive_remote(map_to_rank(bar(B_SFREE + sbuf), 0));
+      if (stop) {
         ab = true;
         break;
       }
@@ -358,16 +450,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       const bool none = (m_run == -INFINITY);
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = none ? 0.f : exp2f(s[2 * c] - m_run);
-        const float p1 = none ? 0.f : exp2f(s[2 * c + 1] - m_run);
+        const float p0 = none ? 0.f : fast_exp2(s[2 * c] - m_run);
+        const float p1 = none ? 0.f : fast_exp2(s[2 * c + 1] - m_run);
         psum += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
       l_part = l_part * alpha + psum;
 
-      // the P buffer is free once PV(j-2) is done
-      if (j >= 2 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + sbuf), ((j - 2) >> 1) & 1);
-      uint8_t* prow = smem + kOffP + sbuf * kPBuf + half * 8192 + row * 128;
+      // the P buffer (and O) are free once PV(j-1) is done
+      if (j >= 1 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
+      uint8_t* prow = smem + kOffP + half * 8192 + row * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 val = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
@@ -376,7 +468,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       // rescale this lane's O row when its running max moved (PV(j-1) must be done)
       const bool warp_need = __any_sync(0xffffffffu, need && j > 0);
       if (warp_need) {
-        if (!ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
         ab = __any_sync(0xffffffffu, ab);
         if (!ab) {
           tc_fence_after();
@@ -395,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(bar(B_PFULL + sbuf), 0));
+      // P(j) of all four warps is written: one arrival for this CTA
+      named_bar_sync(2, 128);
+      if (leader_thread) mbar_arrive_remote(map_to_rank(bar(B_PFULL + sbuf), 0));
     }
 
     // ---------------------------------------------------------------- epilogue
@@ -450,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         } else {
           if (p.rope_tail > 0 && col >= p.Ckv - p.rope_tail) {
             const int pos = len - p.Q + q;
-#pragma unroll 1
+#pragma unroll
             for (int i = 0; i < 16; i += 2) {
               const int jp = (col + i - (p.Ckv - p.rope_tail)) >> 1;
               inverse_rope_pair(f[i], f[i + 1], jp, p.rope_tail, p.rope_theta, pos);
@@ -503,7 +595,7 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
                  const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint32_t elem[3] = {1, 1, 1};
+  cuuint32_t elem[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
                   reinterpret_cast<const cuuint64_t*>(dims),
                   reinterpret_cast<const cuuint64_t*>(strides_bytes),
@@ -568,11 +660,12 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a,
     pe_outer_stride = (uint64_t)a->Lk * a->pe_row_stride * 2;
   }
   {
-    uint64_t d[3] = {512, rows_per, outer};
-    uint64_t s[2] = {(uint64_t)a->kv_row_stride * 2, kv_outer_stride};
-    uint32_t bk[3] = {64, 64, 1}, bv[3] = {64, 32, 1};
-    if (!encode_bf16(&P.tm_k, a->kv_cache, 3, d, s, bk)) return cudaErrorInvalidValue;
-    if (!encode_bf16(&P.tm_v, a->kv_cache, 3, d, s, bv)) return cudaErrorInvalidValue;
+    // (64 dims, rows, 8 chunks of 64 dims, seq|page): a box of 64 rows x 2 chunks
+    // lands as [chunk][row][128 B], two K-major (or MN-major) SW128 blocks
+    uint64_t d[4] = {64, rows_per, 8, outer};
+    uint64_t s[3] = {(uint64_t)a->kv_row_stride * 2, 128, kv_outer_stride};
+    uint32_t bk[4] = {64, 64, 2, 1};
+    if (!encode_bf16(&P.tm_k, a->kv_cache, 4, d, s, bk)) return cudaErrorInvalidValue;
   }
   {
     uint64_t d[3] = {64, rows_per, outer};

@@ -15,6 +15,13 @@ size_t decode_simt_smem(int D);
 cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaStream_t st);
 cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
 
+// tensor-core per-head projections (bf16): B*Q <= 256, Q in {1,2,4}, Dn % 64 == 0, Vd = 128
+bool sm100_proj_supported(int B, int H, int Q, int Dn, int Vd, int Ckv);
+cudaError_t launch_absorb_sm100(const void* q_nope, const void* wkv_b, void* q_lat, int B, int H,
+                                int Q, int Dn, int Vd, int Ckv, cudaStream_t st);
+cudaError_t launch_up_proj_sm100(const void* x, const void* wkv_b, void* out, int B, int H, int Q,
+                                 int Dn, int Vd, int Ckv, cudaStream_t st);
+
 // tensor-core (tcgen05, 2-CTA cluster) decode for bf16, Ckv=512, Dr=64, H*Q % 128 == 0
 bool sm100_decode_supported(const mla_decode_args* a);
 int sm100_auto_splits(const mla_decode_args* a, int sms);
