@@ -42,10 +42,11 @@ using namespace sm100;
 
 constexpr int kThreads = 224;
 constexpr int kTileT = 128;                 // tokens per tile (both CTAs)
-constexpr int kKStages = 5;                 // ring of K stages (16 KB: 2 latent chunks, or rope): a tile
-constexpr int kVStages = 3;                 // ring of V stages (16 KB; a tile uses 4)
-constexpr int kStage = 16384;               // bytes per CTA per stage
-constexpr int kKUses = 5;                   // K stage uses per tile: 4 latent pairs + rope
+constexpr int kKStages = 3;                 // ring of K stages: 3 chunks of 64 dims (24 KB); a tile
+constexpr int kKStage = 24576;
+constexpr int kVStages = 4;                 // ring of V stages (16 KB): a tile
+constexpr int kStage = 16384;               // V stage bytes per CTA
+constexpr int kKUses = 3;                   // K stage uses per tile: chunks 0-2, 3-5, 6-7 + rope
 constexpr int kPrefetchTiles = 0;           // L2 prefetch distance of the K producer (off: measured no gain)
 constexpr int kQBlocks = 9;                 // 64-dim blocks of the 576-wide query row
 constexpr int kQBytes = kQBlocks * 8192;    // 64 rows x 128 B per block
@@ -53,7 +54,7 @@ constexpr int kPBuf = 16384;                // P: 64 rows x 128 tokens bf16 (2 b
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kStage;
+constexpr int kOffV = kOffK + kKStages * kKStage;
 constexpr int kOffP = kOffV + kVStages * kStage;
 constexpr int kOffBar = kOffP + kPBuf;
 enum : int {
@@ -86,6 +87,7 @@ struct alignas(64) Sm100Params {
   CUtensorMap tm_q;    // q_lat  (B*HQ, 512), box 64 x 64
   CUtensorMap tm_qpe;  // q_pe   (B*HQ, 64),  box 64 x 64
   CUtensorMap tm_k;    // latent cache as (64 dims, rows, 8 chunks, seq|page): box 64 rows x 2 chunks
+  CUtensorMap tm_k3;   // the same view, box 64 rows x 3 chunks
   CUtensorMap tm_pe;   // rope cache (64 dims, rows, seq|page): box 64 rows
   DecodeParams p;
   int paged;
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       tma_prefetch_desc(&P.tm_q);
       tma_prefetch_desc(&P.tm_qpe);
       tma_prefetch_desc(&P.tm_k);
+      tma_prefetch_desc(&P.tm_k3);
       tma_prefetch_desc(&P.tm_pe);
       const int qrow = b * p.HQ + rb * 128 + (int)rank * 64;
       const uint32_t qbar = map_to_rank(bar(B_QFULL), 0);
@@ -238,13 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         for (int u = 0; u < kKUses; ++u, ++it) {
           const uint32_t s = it % kKStages, round = it / kKStages;
           if (round > 0 && !mbar_wait_cluster(bar(B_KEMPTY + s), (round - 1) & 1)) { ok = false; break; }
-          const uint32_t dst = sb0 + kOffK + s * kStage, fb = map_to_rank(bar(B_KFULL + s), 0);
-          if (u < 4) {
-            if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * kStage);
-            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 2 * u, zc);
+          const uint32_t dst = sb0 + kOffK + s * kKStage, fb = map_to_rank(bar(B_KFULL + s), 0);
+          if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * kKStage);
+          if (u < 2) {
+            tma_load_4d_2sm(dst, &P.tm_k3, fb, 0, y, 3 * u, zc);
           } else {
-            if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * 8192);
-            tma_load_3d_2sm(dst, &P.tm_pe, fb, 0, y, zc);
+            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 6, zc);
+            tma_load_3d_2sm(dst + 2 * 8192, &P.tm_pe, fb, 0, y, zc);
           }
         }
         if (*abort_flag) ok = false;
@@ -311,10 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
           if (sfree && mbar_poll_cluster(bar(B_KFULL + s), (kit / kKStages) & 1)) {
             tc_fence_after();
             const uint32_t d = tmem + kColS + 64u * sbuf;
-            const uint32_t kb = sb0 + kOffK + s * kStage;
-            const int nch = (qu < 4) ? 2 : 1;
-            for (int cc = 0; cc < nch; ++cc) {
-              const int c = (qu < 4) ? 2 * qu + cc : 8;   // 64-dim block of Q
+            const uint32_t kb = sb0 + kOffK + s * kKStage;
+            for (int cc = 0; cc < 3; ++cc) {
+              const int c = 3 * qu + cc;                  // 64-dim block of Q (8 = rope)
               const uint32_t qa = sb0 + kOffQ + c * 8192, ka = kb + cc * 8192;
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
@@ -664,8 +666,9 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a,
     // lands as [chunk][row][128 B], two K-major (or MN-major) SW128 blocks
     uint64_t d[4] = {64, rows_per, 8, outer};
     uint64_t s[3] = {(uint64_t)a->kv_row_stride * 2, 128, kv_outer_stride};
-    uint32_t bk[4] = {64, 64, 2, 1};
+    uint32_t bk[4] = {64, 64, 2, 1}, bk3[4] = {64, 64, 3, 1};
     if (!encode_bf16(&P.tm_k, a->kv_cache, 4, d, s, bk)) return cudaErrorInvalidValue;
+    if (!encode_bf16(&P.tm_k3, a->kv_cache, 4, d, s, bk3)) return cudaErrorInvalidValue;
   }
   {
     uint64_t d[3] = {64, rows_per, outer};
