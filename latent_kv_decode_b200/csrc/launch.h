@@ -15,8 +15,10 @@ size_t decode_simt_smem(int D);
 cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaStream_t st);
 cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
 
-// tensor-core per-head projections (bf16): B*Q <= 256, Q in {1,2,4}, Dn % 64 == 0, Vd = 128
-bool sm100_proj_supported(int B, int H, int Q, int Dn, int Vd, int Ckv);
+// tensor-core per-head projections (bf16): Ckv = 512, Vd = 128, Dn in {64, 128}, 16-byte
+// aligned activation, weight and output pointers
+bool sm100_proj_supported(int B, int H, int Q, int Dn, int Vd, int Ckv, const void* act,
+                          const void* w, const void* out);
 cudaError_t launch_absorb_sm100(const void* q_nope, const void* wkv_b, void* q_lat, int B, int H,
                                 int Q, int Dn, int Vd, int Ckv, cudaStream_t st);
 cudaError_t launch_up_proj_sm100(const void* x, const void* wkv_b, void* out, int B, int H, int Q,

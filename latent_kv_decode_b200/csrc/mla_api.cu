@@ -192,7 +192,7 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* wkv_b, void* q_lat, in
   mla_status_t s = check_proj(q_nope, wkv_b, q_lat, B, H, Q, Dn, Vd, Ckv, dt);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (dt == MLA_BF16 && mla::sm100_proj_supported(B, H, Q, Dn, Vd, Ckv))
+  if (dt == MLA_BF16 && mla::sm100_proj_supported(B, H, Q, Dn, Vd, Ckv, q_nope, wkv_b, q_lat))
     return cuda_status(mla::launch_absorb_sm100(q_nope, wkv_b, q_lat, B, H, Q, Dn, Vd, Ckv, st));
   return cuda_status(
       mla::launch_absorb_simt(q_nope, wkv_b, q_lat, B, H, Q, Dn, Vd, Ckv, dt == MLA_BF16, st));
@@ -203,7 +203,7 @@ mla_status_t mla_up_proj(const void* x, const void* wkv_b, void* out, int B, int
   mla_status_t s = check_proj(x, wkv_b, out, B, H, Q, Dn, Vd, Ckv, dt);
   if (s != MLA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  if (dt == MLA_BF16 && mla::sm100_proj_supported(B, H, Q, Dn, Vd, Ckv))
+  if (dt == MLA_BF16 && mla::sm100_proj_supported(B, H, Q, Dn, Vd, Ckv, x, wkv_b, out))
     return cuda_status(mla::launch_up_proj_sm100(x, wkv_b, out, B, H, Q, Dn, Vd, Ckv, st));
   return cuda_status(
       mla::launch_up_proj_simt(x, wkv_b, out, B, H, Q, Dn, Vd, Ckv, dt == MLA_BF16, st));

@@ -3,19 +3,23 @@
 //   mla_absorb_q  blank [1] of the 6547.cn MLA decode question:
 //                 q_lat[b,h,q,c] = sum_d q_nope[b,h,q,d] W_UK[h][d][c]
 //                 computed transposed, D[c][n] = W_UK[h]^T . q_nope[n]^T:
-//                 M = 128 latent columns per CTA (A = W_UK, MN-major),
-//                 N = B*Q query rows, K = Dn.
+//                 4 M tiles of 128 latent columns (A = W_UK, MN-major),
+//                 N = query rows n = (b, q), K = Dn.
 //   mla_up_proj   blank [5]: out[b,h,q,v] = sum_c x[b,h,q,c] W_UV[h][v][c]
 //                 D[v][n] = W_UV[h] . x[n]^T: M = Vd = 128 (A = W_UV,
-//                 K-major), N = B*Q, K = Ckv = 512.
+//                 K-major), N = query rows, K = Ckv = 512.
 //
-// One CTA per (head, 128-row M tile). K is walked in 64-wide blocks through a
-// ring of shared-memory stages filled by TMA (warp 0) and consumed by single-
-// thread tcgen05.mma issue (warp 1); D (128 lanes x N fp32 columns) lives in
-// TMEM and all four warps write it out. Both ops stream their weight (16.8 MB
-// at H=128) once, so they are HBM-bound; N = B*Q <= 256.
-#include <cudaTypedefs.h>
-
+// One CTA per (head, block of up to 64 query rows); absorb also splits the
+// 512 latent columns into two CTAs (two CTAs per SM, all SMs busy). Both ops
+// stream a 128 KB weight slice per head (16.8 MB at H = 128) and are
+// HBM-bound, so the CTA issues every 16-byte load of its slice and of its
+// activation rows at once (512 threads; a warp reads 512 contiguous bytes of a
+// weight row; at most 192 KB in flight), stores them into the 128-byte-
+// swizzled layouts the MMAs read, and one thread then issues the tcgen05 MMAs
+// (K = 16 each) into TMEM. 16 warps move D through shared memory, transposed
+// to query rows, and write whole output rows with 16-byte stores. Plain loads
+// rather than TMA boxes: a box of 64 columns reads 128 B of every 1 KB weight
+// row, eight passes over the same DRAM rows per head.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100_ptx.cuh"
@@ -25,229 +29,257 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kPThreads = 128;
-constexpr int kPStages = 4;
-constexpr int kMaxN = 256;
+constexpr int kPThreads = 512;
+constexpr int kRowsPerCta = 64;    // query rows (MMA N) per CTA
+constexpr int kWUnits = 64;        // 16-byte units per weight row (Ckv = 512)
+// 16-byte loads per thread: absorb (128 rows x 512 B + 64 rows x 256 B) / 512,
+// up (128 + 64 rows x 1 KB) / 512
+template <bool kAbsorb>
+constexpr int kPieces = kAbsorb ? 10 : 24;
 
-struct alignas(64) ProjParams {
-  CUtensorMap tm_a;   // weight
-  CUtensorMap tm_b;   // query / latent rows (D, Q, H, B)
-  void* out;
-  int B, H, Q, N;     // N = B*Q rounded up to a multiple of 16
-  int nkb;            // 64-wide K blocks
-  int a_mn_major;     // absorb: W_UK read M-major; up: W_UV read K-major
-  int row0;           // first weight row of the head's slice (0 for W_UK, Dn for W_UV)
-  int out_cols;       // columns per output row: 512 (q_lat) or Vd (out)
-  int a_bytes, b_bytes;  // per stage
+struct ProjArgs {
+  const __nv_bfloat16* act;   // q_nope (B,H,Q,Dn) or x (B,H,Q,Ckv)
+  const __nv_bfloat16* w;     // wkv_b (H, Dn+Vd, Ckv)
+  __nv_bfloat16* out;         // q_lat (B,H,Q,Ckv) or out (B,H,Q,Vd)
+  int H, Q, rows;             // rows = B*Q
+  int w_head_rows;            // Dn + Vd
+  int w_row0;                 // first row of the head's slice: 0 (W_UK) or Dn (W_UV)
+  int w_rows;                 // rows of the slice: Dn or Vd
+  int K;                      // reduction length: Dn (absorb) or Ckv (up)
+  int out_cols;               // Ckv (absorb) or Vd (up)
+  int w_units;                // 16-byte units of each weight row loaded per CTA: 32 (absorb) or 64
+  int absorb;
   int32_t* err;
 };
 
-__global__ void __launch_bounds__(kPThreads, 1) proj_sm100_kernel(const __grid_constant__ ProjParams P) {
+// Element offset of query row n = b*Q + q of head h in a (B, H, Q, cols) tensor.
+__device__ __forceinline__ int64_t row_off(int n, int h, int H, int Q, int cols) {
+  const int b = n / Q, q = n - b * Q;
+  return (((int64_t)b * H + h) * Q + q) * cols;
+}
+
+// Byte offset of 16-byte unit u of row r in a stack of 128-byte-swizzled
+// blocks: block u/8 holds units [8(u/8), 8(u/8)+8) of every row.
+__device__ __forceinline__ uint32_t sw128_off(int r, int u, uint32_t block_bytes) {
+  return (uint32_t)(u >> 3) * block_bytes + (uint32_t)r * 128u +
+         ((uint32_t)((u & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+template <bool kAbsorb>
+__global__ void __launch_bounds__(kPThreads, kAbsorb ? 2 : 1) proj_sm100_kernel(const ProjArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb0 = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sb0 - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x, mt = blockIdx.y;
-  const int stage_bytes = P.a_bytes + P.b_bytes;
-  const uint32_t off_bar = kPStages * stage_bytes;
-  auto bar = [&](int i) -> uint32_t { return sb0 + off_bar + 8u * (uint32_t)i; };
-  // bars: full[4], empty[4], done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * kPStages + 1));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + off_bar + 8 * (2 * kPStages + 1) + 4);
+  const int h = blockIdx.x;
+  const int col_half = blockIdx.y;                // absorb: latent columns [256 col_half, +256)
+  const int n0 = blockIdx.z * kRowsPerCta;
+  const int nrows = min(kRowsPerCta, a.rows - n0);
+  const int N = (nrows + 15) & ~15;               // MMA N: a multiple of 16
+
+  // shared layout: weight slice (w_units/8 blocks of 64 columns x w_rows) |
+  // activation rows (K/64 blocks x N rows) | done barrier, TMEM slot. After the
+  // MMAs the weight area holds the transposed output rows.
+  const int w_units = a.w_units;
+  const int w_ushift = 31 - __clz(w_units);
+  const uint32_t w_block = (uint32_t)a.w_rows * 128u;
+  const uint32_t off_x = (uint32_t)(w_units >> 3) * w_block;
+  const int a_units = a.K >> 3;                   // 16-byte units per activation row
+  const uint32_t x_block = (uint32_t)N * 128u;
+  const uint32_t off_bar = off_x + (uint32_t)(a_units >> 3) * x_block;
+  const uint32_t bar_done = sb0 + off_bar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8);
+  const int m_tiles = kAbsorb ? 2 : 1;           // absorb: 256 latent columns = 2 M tiles
+  const uint32_t tmem_cols = kAbsorb ? 128u : 64u;  // m_tiles x N (<= 64)
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPStages; ++s) {
-      mbar_init(bar(s), 1);
-      mbar_init(bar(kPStages + s), 1);
-    }
-    mbar_init(bar(2 * kPStages), 1);
-    *abort_flag = 0;
+    mbar_init(bar_done, 1);
     fence_mbar_init();
   }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
+
+  // ---------------------------------------------------------------- loads
+  // piece p < nw: unit p % w_units of weight row p / w_units; then unit
+  // q % a_units of activation row q / a_units (q = p - nw). All issued before
+  // any store.
+  const int nw = a.w_rows * w_units;
+  const int np = nw + nrows * a_units;
+  const int a_shift = 31 - __clz(a_units);        // a_units is a power of two
+  const char* wslice = reinterpret_cast<const char*>(
+      a.w + ((int64_t)h * a.w_head_rows + a.w_row0) * (kWUnits * 8) + col_half * (w_units * 8));
+  uint4 v[kPieces<kAbsorb>];
+#pragma unroll
+  for (int i = 0; i < kPieces<kAbsorb>; ++i) {
+    const int p = (int)threadIdx.x + i * kPThreads;
+    if (p < nw) {
+      const int r = p >> w_ushift, u = p & (w_units - 1);
+      v[i] = ld_stream(wslice + (int64_t)r * (kWUnits * 16) + u * 16);
+    } else if (p < np) {
+      const int q = p - nw, r = q >> a_shift, u = q & (a_units - 1);
+      v[i] = ld_stream(a.act + row_off(n0 + r, h, a.H, a.Q, a.K) + u * 8);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kPieces<kAbsorb>; ++i) {
+    const int p = (int)threadIdx.x + i * kPThreads;
+    if (p < nw) {
+      const int r = p >> w_ushift, u = p & (w_units - 1);
+      *reinterpret_cast<uint4*>(smem + sw128_off(r, u, w_block)) = v[i];
+    } else if (p < np) {
+      const int q = p - nw, r = q >> a_shift, u = q & (a_units - 1);
+      *reinterpret_cast<uint4*>(smem + off_x + sw128_off(r, u, x_block)) = v[i];
+    }
+  }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
-  auto fail = [&]() {
-    *abort_flag = 1;
-    if (P.err) atomicOr(P.err, MLA_DEVICE_ERR_TIMEOUT);
-  };
 
-  if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    for (int kb = 0; kb < P.nkb; ++kb) {
-      const int s = kb % kPStages;
-      if (kb >= kPStages && !mbar_wait(bar(kPStages + s), ((kb / kPStages) - 1) & 1)) {
-        fail();
-        break;
-      }
-      const uint32_t a_dst = sb0 + s * stage_bytes, b_dst = a_dst + P.a_bytes;
-      mbar_arrive_expect_tx(bar(s), P.a_bytes + P.b_bytes);
-      if (P.a_mn_major) {
-        // W_UK[h] rows d in [64 kb, 64 kb + 64), columns c in this M tile: two 64-wide MN blocks
-        tma_load_3d(a_dst, &P.tm_a, bar(s), 128 * mt, P.row0 + 64 * kb, h);
-        tma_load_3d(a_dst + 8192, &P.tm_a, bar(s), 128 * mt + 64, P.row0 + 64 * kb, h);
-      } else {
-        // W_UV[h] rows v (128), columns c in [64 kb, 64 kb + 64)
-        tma_load_3d(a_dst, &P.tm_a, bar(s), 64 * kb, P.row0, h);
-      }
-      // query rows n = (b, q) of head h, K columns [64 kb, 64 kb + 64)
-      asm volatile(
-          "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-          " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(b_dst),
-          "l"(reinterpret_cast<uint64_t>(&P.tm_b)), "r"(bar(s)), "r"(64 * kb), "r"(0), "r"(h), "r"(0)
-          : "memory");
+  // ---------------------------------------------------------------- MMAs
+  // lane 0 of warp 0 issues; the warp reconverges before anyone waits on D
+  if (threadIdx.x == 0) {
+    const int ksteps = a.K >> 4;
+    if (kAbsorb) {
+      // D[c][n], M tile mt = latent columns [128 mt, 128 mt + 128) of this
+      // CTA's half: A = two 64-column blocks of W_UK (MN-major, rows d),
+      // B = q_nope rows (K-major)
+      const uint32_t idesc = idesc_bf16_f32(128, N, true, false);
+      for (int mt = 0; mt < m_tiles; ++mt)
+        for (int ks = 0; ks < ksteps; ++ks)
+          mma_bf16_ss(tmem + (uint32_t)(mt * N),
+                      smem_desc(sb0 + 2u * mt * w_block + 2048u * ks, w_block, 1024, kSwizzle128B),
+                      smem_desc(sb0 + off_x + (ks >> 2) * x_block + 32u * (ks & 3), 16, 1024,
+                                kSwizzle128B),
+                      idesc, ks > 0);
+    } else {
+      // D[v][n]: A = W_UV rows v (K-major), B = x rows (K-major)
+      const uint32_t idesc = idesc_bf16_f32(128, N, false, false);
+      for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16_ss(tmem,
+                    smem_desc(sb0 + (ks >> 2) * w_block + 32u * (ks & 3), 16, 1024, kSwizzle128B),
+                    smem_desc(sb0 + off_x + (ks >> 2) * x_block + 32u * (ks & 3), 16, 1024,
+                              kSwizzle128B),
+                    idesc, ks > 0);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_bf16_f32(128, P.N, P.a_mn_major != 0, false);
-    bool ok = true;
-    for (int kb = 0; kb < P.nkb && ok; ++kb) {
-      const int s = kb % kPStages;
-      if (!mbar_wait(bar(s), (kb / kPStages) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t a = sb0 + s * stage_bytes, bb = a + P.a_bytes;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t ad = P.a_mn_major ? smem_desc(a + 2048 * k, 8192, 1024, kSwizzle128B)
-                                         : smem_desc(a + 32 * k, 16, 1024, kSwizzle128B);
-        mma_bf16_ss(tmem, ad, smem_desc(bb + 32 * k, 16, 1024, kSwizzle128B), idesc,
-                    (kb | k) != 0);
-      }
-      mma_commit(bar(kPStages + s));
-    }
-    if (ok) mma_commit(bar(2 * kPStages));
-    else fail();
+    mma_commit(bar_done);
   }
   __syncwarp();
 
-  // ------------------------------------------------------------------ epilogue
-  bool ok = mbar_wait(bar(2 * kPStages), 0);
+  // ---------------------------------------------------------------- epilogue
+  // D row m (TMEM lane 32*quadrant + lane of M tile mt) is output column
+  // 128 mt + m of the CTA's columns; D column n is query row n. Warp
+  // 4 * part + quadrant moves its lanes' columns [c_lo, c_hi) into rows n of
+  // a bf16 staging tile (row pitch = the CTA's output columns), then the CTA
+  // writes whole rows.
+  bool ok = mbar_wait(bar_done, 0);
   ok = __all_sync(0xffffffffu, ok) != 0;
   tc_fence_after();
-  const int m = 32 * warp + lane;                       // TMEM lane = output column within the tile
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-  const int rows = P.B * P.Q;
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
-  const int col = 128 * mt + m;
+  const int g = warp & 3, part = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(32 * g) << 16;
+  const int ocols = 128 * m_tiles;                // output columns of this CTA
+  __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);
   if (ok) {
-    for (int n0 = 0; n0 < P.N; n0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + (uint32_t)n0, v);
+    int mt, c_lo, c_hi;
+    if (kAbsorb) {                               // 2 M tiles x 2 column halves of N
+      mt = part & 1;
+      const int hn = ((N >> 1) + 15) & ~15;
+      c_lo = min((part >> 1) * hn, N);
+      c_hi = (part >> 1) ? N : min(hn, N);
+    } else {                                      // 1 M tile x 4 column quarters of N
+      mt = 0;
+      c_lo = min(part * 16, N);
+      c_hi = min(c_lo + 16, N);
+    }
+    const int m = 128 * mt + 32 * g + lane;
+    for (int c = c_lo; c < c_hi; c += 16) {
+      uint32_t d[16];
+      tmem_ld16(tmem + lane_base + (uint32_t)(mt * N + c), d);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int n = n0 + i;
-        if (n < rows) {
-          const int b = n / P.Q, q = n % P.Q;
-          out[(((int64_t)b * P.H + h) * P.Q + q) * P.out_cols + col] =
-              __float2bfloat16_rn(__uint_as_float(v[i]));
-        }
-      }
+      for (int i = 0; i < 16; ++i) stage[(c + i) * ocols + m] = __float2bfloat16_rn(__uint_as_float(d[i]));
     }
-  } else if (threadIdx.x == 0) {
-    fail();
+  } else if (threadIdx.x == 0 && a.err) {
+    atomicOr(a.err, MLA_DEVICE_ERR_TIMEOUT);
+  }
+  __syncthreads();
+  if (ok) {
+    const int upr = ocols >> 3;                   // 16-byte units per staged row
+    const int col0 = kAbsorb ? 256 * col_half : 0;
+    for (int e = threadIdx.x; e < nrows * upr; e += kPThreads) {
+      const int n = e / upr, u = e - n * upr;
+      *reinterpret_cast<uint4*>(a.out + row_off(n0 + n, h, a.H, a.Q, a.out_cols) + col0 + u * 8) =
+          *reinterpret_cast<const uint4*>(stage + n * ocols + u * 8);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, tmem_cols);
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 proj_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-bool proj_encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box) {
-  auto fn = proj_encode_fn();
-  if (!fn) return false;
-  cuuint32_t elem[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-            reinterpret_cast<const cuuint64_t*>(dims),
-            reinterpret_cast<const cuuint64_t*>(strides_bytes),
-            reinterpret_cast<const cuuint32_t*>(box), elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// rows: (K, Q, H, B) view of a (B, H, Q, K) tensor; box 64 x Q x 1 x ceil(N/Q)
-bool encode_rows(CUtensorMap* m, const void* base, int B, int H, int Q, int K, int N) {
-  uint64_t d[4] = {(uint64_t)K, (uint64_t)Q, (uint64_t)H, (uint64_t)B};
-  uint64_t s[3] = {(uint64_t)K * 2, (uint64_t)Q * K * 2, (uint64_t)H * Q * K * 2};
-  uint32_t box[4] = {64, (uint32_t)Q, 1, (uint32_t)((N + Q - 1) / Q)};
-  return proj_encode(m, base, 4, d, s, box);
+size_t proj_smem_bytes(bool absorb, int Dn, int Vd, int Ckv) {
+  const int w_rows = absorb ? Dn : Vd;
+  const int K = absorb ? Dn : Ckv;
+  const int w_blocks = absorb ? 4 : 8;
+  return (size_t)w_blocks * w_rows * 128 + (size_t)(K / 64) * kRowsPerCta * 128 + 64 + 1024;
 }
 
 cudaError_t launch_proj(bool absorb, const void* act, const void* w, void* out, int B, int H, int Q,
                         int Dn, int Vd, int Ckv, cudaStream_t st) {
-  ProjParams P;
-  memset(&P, 0, sizeof(P));
-  const int rows = B * Q;
-  P.out = out;
-  P.B = B;
-  P.H = H;
-  P.Q = Q;
-  P.N = ((rows + 15) / 16) * 16;           // a multiple of 16, hence of Q in {1, 2, 4}
-  const int K = absorb ? Dn : Ckv;
-  P.nkb = K / 64;
-  P.b_bytes = P.N * 128;
-  uint64_t wd[3] = {(uint64_t)Ckv, (uint64_t)(Dn + Vd), (uint64_t)H};
-  uint64_t ws[2] = {(uint64_t)Ckv * 2, (uint64_t)(Dn + Vd) * Ckv * 2};
-  if (absorb) {
-    P.a_mn_major = 1;
-    P.row0 = 0;
-    P.out_cols = Ckv;
-    P.a_bytes = 2 * 8192;                  // 64 K rows x 2 MN blocks of 128 B
-    uint32_t box[3] = {64, 64, 1};
-    if (!proj_encode(&P.tm_a, w, 3, wd, ws, box)) return cudaErrorInvalidValue;
-  } else {
-    P.a_mn_major = 0;
-    P.row0 = Dn;
-    P.out_cols = Vd;
-    P.a_bytes = 128 * 128;                 // 128 M rows x 64 K columns
-    uint32_t box[3] = {64, 128, 1};
-    if (!proj_encode(&P.tm_a, w, 3, wd, ws, box)) return cudaErrorInvalidValue;
-  }
-  if (!encode_rows(&P.tm_b, act, B, H, Q, K, P.N)) return cudaErrorInvalidValue;
-  const int smem = kPStages * (P.a_bytes + P.b_bytes) + 1024 + 1024;
-  cudaError_t e = cudaFuncSetAttribute(proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  ProjArgs a;
+  a.act = reinterpret_cast<const __nv_bfloat16*>(act);
+  a.w = reinterpret_cast<const __nv_bfloat16*>(w);
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.H = H;
+  a.Q = Q;
+  a.rows = B * Q;
+  a.w_head_rows = Dn + Vd;
+  a.w_row0 = absorb ? 0 : Dn;
+  a.w_rows = absorb ? Dn : Vd;
+  a.K = absorb ? Dn : Ckv;
+  a.out_cols = absorb ? Ckv : Vd;
+  a.w_units = absorb ? 32 : 64;
+  a.absorb = absorb ? 1 : 0;
+  a.err = nullptr;
+  const int smem = (int)proj_smem_bytes(absorb, Dn, Vd, Ckv);
+  auto kern = absorb ? proj_sm100_kernel<true> : proj_sm100_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(H, absorb ? Ckv / 128 : Vd / 128);
-  proj_sm100_kernel<<<grid, kPThreads, smem, st>>>(P);
+  dim3 grid(H, absorb ? 2 : 1, (a.rows + kRowsPerCta - 1) / kRowsPerCta);
+  kern<<<grid, kPThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-bool sm100_proj_supported(int B, int H, int Q, int Dn, int Vd, int Ckv) {
-  const int rows = B * Q;
-  if (rows < 1 || rows > kMaxN || !(Q == 1 || Q == 2 || Q == 4)) return false;
-  if (Dn % 64 != 0 || Vd != 128 || Ckv != 512) return false;
+bool sm100_proj_supported(int B, int H, int Q, int Dn, int Vd, int Ckv, const void* act,
+                          const void* w, const void* out) {
+  if (B < 1 || H < 1 || Q < 1) return false;
+  // Ckv = 512 (8 blocks of 64), Vd = 128 (one M tile), Dn in {64, 128}: the
+  // whole slice and 64 rows fit in shared memory and in 24 loads per thread
+  if (Ckv != 512 || Vd != 128 || !(Dn == 64 || Dn == 128)) return false;
+  const auto aligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!aligned(act) || !aligned(w) || !aligned(out)) return false;
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
     return false;
-  return major == 10 && proj_encode_fn() != nullptr;
+  return major == 10;
 }
 
 cudaError_t launch_absorb_sm100(const void* q_nope, const void* wkv_b, void* q_lat, int B, int H,

@@ -32,6 +32,23 @@ def _check_step(w, g, batch=None, tol=None, rel=None):
     assert_close(g["out"][sel], ref["out"], tol, "out(end to end)", rel)
 
 
+@pytest.mark.parametrize("B,Q,Dn", [(70, 1, 128), (33, 2, 128), (5, 4, 64), (1, 1, 128)])
+def test_projections_row_blocks(B, Q, Dn):
+    """Both projections on their own: query rows in blocks of 64 with a ragged
+    last block (70, 66, 20 and 1 rows), Q > 1 and Dn = 64. up_proj is fed the
+    GPU's q_lat as its latent input."""
+    from latent_kv_decode_b200 import ops
+    w = wl.make_mla(B=B, H=8, Q=Q, Dn=Dn, Dr=64, Vd=128, Ckv=512, Lk=8, dtype="bf16", seed=11)
+    d = upload(w)
+    q_lat = ops.mla_absorb_q(d["q_nope"], d["wkv_b"])
+    out = ops.mla_up_proj(q_lat, d["wkv_b"], Dn)
+    torch.cuda.synchronize()
+    g_lat = q_lat.float().cpu().numpy().astype(np.float64)
+    g_out = out.float().cpu().numpy().astype(np.float64)
+    assert_close(g_lat, omla.absorb_q(w.q_nope, w.wkv_b), TOL_BF16, "q_lat", REL_L2_BF16)
+    assert_close(g_out, omla.up_proj(g_lat, w.wkv_b, Dn), TOL_BF16, "out", REL_L2_BF16)
+
+
 @pytest.mark.parametrize("splits", [0, 1, 3])
 def test_demo_fp32(splits):
     w = wl.demo_fp32()
