@@ -68,6 +68,23 @@ def make_workload(name: str, rank: int):
     raise SystemExit(f"unknown workload {name}")
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank floats across the process group (every
+    rank gets the result); identity without a group."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(B: int, Q: int, world: int, step_ms: float) -> float:
+    """Whole-job throughput: every rank decodes its own B*Q query rows per step
+    (weak scaling), so the job does B*Q*world rows per max-over-ranks step."""
+    return B * Q * world / (step_ms * 1e-3)
+
+
 def workload_desc(w) -> dict:
     d = dict(workload=f"{w.name}: B={w.B} H={w.H} Q={w.Q} Dn={w.Dn} Dr={w.Dr} Vd={w.Vd} "
                       f"Ckv={w.Ckv} Lk={w.Lk}{' ragged paged' if w.block_table is not None else ''}"
@@ -292,10 +309,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     e2e_mean = sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / K
 
-    stats = torch.tensor([mean_step, mean_dec, e2e_mean], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    mean_step, mean_dec, e2e_mean = stats.tolist()
+    mean_step, mean_dec, e2e_mean = max_over_ranks([mean_step, mean_dec, e2e_mean], dist, dev)
     if rank != 0:
         return None
 
@@ -308,7 +322,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     step_tf = alg["step_flops"] / (mean_step * 1e-3) / 1e12
     roof_s = max(alg["step_bytes"] / (hbm * 1e9), alg["step_flops"] / (tflops * 1e12))
     tokens = w.B * w.Q * world
-    value = tokens / (mean_step * 1e-3)
+    value = job_tokens_per_s(w.B, w.Q, world, mean_step)
     pct = lambda xs, q: float(np.percentile(np.asarray(xs), q))
     res = {
         "metric": METRIC,
@@ -348,7 +362,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                           "combine": round(sum(comb_ms) / K, 5), "up_proj": round(sum(up_ms) / K, 5)},
         },
         "e2e": {
-            "value": round(tokens / (e2e_mean * 1e-3), 1), "unit": "tokens/s",
+            "value": round(job_tokens_per_s(w.B, w.Q, world, e2e_mean), 1), "unit": "tokens/s",
             "ms_per_step": round(e2e_mean, 5),
             "h2d_bytes_per_step": int(q_nope.numel() * q_nope.element_size() +
                                       q_pe.numel() * q_pe.element_size()),
