@@ -1,0 +1,31 @@
+"""Host-side pieces of bench.py that need no GPU: the clock summary and the
+algorithmic byte / flop counts the roofline divides by."""
+import bench
+from latent_kv_decode_b200 import workloads as wl
+
+
+def test_clock_summary_maps_nvml_reason_bits():
+    c = bench.ClockSampler(0)
+    c.samples = [(1965.0, 1965.0, 0x0), (1900.0, 1965.0, 0x4), (1305.0, 1965.0, 0x8 | 0x40)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_clock_summary_reads_nvidia_smi_lines():
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_algorithmic_bytes_of_the_dsv3_step():
+    # cache (B*Lk*(Ckv+Dr)*2) + wkv_b (H*(Dn+Vd)*Ckv*2) + q (B*H*(Dn+Dr)*2) + out (B*H*Vd*2)
+    w = wl.Workload(name="shape", B=64, H=128, Q=1, Dn=128, Dr=64, Vd=128, Ckv=512, Lk=4096,
+                    dtype="bf16", softmax_scale=1.0, q_nope=None, q_pe=None, kv_cache=None,
+                    pe_cache=None, wkv_b=None)
+    a = bench.algorithmic(w)
+    assert a["step_bytes"] == 64 * 4096 * 576 * 2 + 128 * 256 * 512 * 2 + 64 * 128 * 192 * 2 + 64 * 128 * 128 * 2
+    assert a["step_bytes"] == 340_787_200
+    # QK 576-wide + PV 512-wide per (row, token); absorb + up-projection per row
+    assert a["step_flops"] == 2 * 64 * 128 * 4096 * (576 + 512) + 2 * 64 * 128 * 512 * (128 + 128)
