@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int rb = blockIdx.x >> 1, b = blockIdx.y, z = blockIdx.z;
+  pdl_launch_dependents();
   const int len = seq_len_of(p, b);
   int t_begin, t_end;
   split_range(len, p.num_splits, z, t_begin, t_end);
@@ -202,6 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       tma_prefetch_desc(&P.tm_k);
       tma_prefetch_desc(&P.tm_k3);
       tma_prefetch_desc(&P.tm_pe);
+      // q_lat comes from the previous kernel (the absorb): read it only once
+      // that grid has completed; everything above overlapped its tail
+      pdl_wait();
       const int qrow = b * p.HQ + rb * 128 + (int)rank * 64;
       const uint32_t qbar = map_to_rank(bar(B_QFULL), 0);
       if (rank == 0) mbar_arrive_expect_tx(bar(B_QFULL), 2 * kQBytes);
@@ -684,13 +688,15 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a,
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemAlloc;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, decode_sm100_kernel, P);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

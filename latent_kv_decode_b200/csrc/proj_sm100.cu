@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kPThreads, kAbsorb ? 2 : 1) proj_sm100_kernel(
   const int m_tiles = kAbsorb ? 2 : 1;           // absorb: 256 latent columns = 2 M tiles
   const uint32_t tmem_cols = kAbsorb ? 128u : 64u;  // m_tiles x N (<= 64)
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     mbar_init(bar_done, 1);
     fence_mbar_init();
@@ -119,10 +120,17 @@ __global__ void __launch_bounds__(kPThreads, kAbsorb ? 2 : 1) proj_sm100_kernel(
   const int a_shift = 31 - __clz(a_units);        // a_units is a power of two
   const char* wslice = reinterpret_cast<const char*>(
       a.w + ((int64_t)h * a.w_head_rows + a.w_row0) * (kWUnits * 8) + col_half * (w_units * 8));
+  // the weight slice is a read-only input: it streams in while the previous
+  // kernel finishes; the activation rows are read only after pdl_wait()
   uint4 v[kPieces<kAbsorb>];
+  bool waited = false;
 #pragma unroll
   for (int i = 0; i < kPieces<kAbsorb>; ++i) {
     const int p = (int)threadIdx.x + i * kPThreads;
+    if (p >= nw && !waited) {   // the same i for every thread: nw is a multiple of 512
+      pdl_wait();
+      waited = true;
+    }
     if (p < nw) {
       const int r = p >> w_ushift, u = p & (w_units - 1);
       v[i] = ld_stream(wslice + (int64_t)r * (kWUnits * 16) + u * 16);
@@ -142,6 +150,7 @@ __global__ void __launch_bounds__(kPThreads, kAbsorb ? 2 : 1) proj_sm100_kernel(
       *reinterpret_cast<uint4*>(smem + off_x + sw128_off(r, u, x_block)) = v[i];
     }
   }
+  if (!waited) pdl_wait();
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -260,8 +269,18 @@ cudaError_t launch_proj(bool absorb, const void* act, const void* w, void* out, 
   auto kern = absorb ? proj_sm100_kernel<true> : proj_sm100_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(H, absorb ? 2 : 1, (a.rows + kRowsPerCta - 1) / kRowsPerCta);
-  kern<<<grid, kPThreads, smem, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(H, absorb ? 2 : 1, (a.rows + kRowsPerCta - 1) / kRowsPerCta);
+  cfg.blockDim = dim3(kPThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
