@@ -65,6 +65,8 @@ def make_workload(name: str, rank: int):
         return wl.longctx(seed=3 + 1000 * rank)
     if name == "ragged_paged_b128_q2":
         return wl.ragged_paged(seed=2 + 1000 * rank)
+    if name == "v41_fp4_sink_h64":
+        return wl.v41_shared_latent(seed=4 + 1000 * rank)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -86,6 +88,12 @@ def job_tokens_per_s(B: int, Q: int, world: int, step_ms: float) -> float:
 
 
 def workload_desc(w) -> dict:
+    if w.q is not None:
+        return dict(workload=f"{w.name}: B={w.B} H={w.H} Q={w.Q} Ckv={w.Ckv} Lk={w.Lk}, shared latent "
+                             f"(K = V), FP4 E2M1 with an E4M3 scale per 16 (288 B/token), sink, "
+                             f"inverse RoPE on the last {w.rope_tail} dims, bf16 q and x",
+                    B=w.B, H=w.H, Q=w.Q, Lk=w.Lk, Ckv=w.Ckv, cache="contiguous FP4 entries",
+                    l2="flushed before every timed step (256 MiB write)")
     d = dict(workload=f"{w.name}: B={w.B} H={w.H} Q={w.Q} Dn={w.Dn} Dr={w.Dr} Vd={w.Vd} "
                       f"Ckv={w.Ckv} Lk={w.Lk}{' ragged paged' if w.block_table is not None else ''}"
                       f", {w.dtype} storage, fp32 accumulate",
@@ -106,6 +114,15 @@ def algorithmic(w):
     """
     es = 4 if w.dtype == "f32" else 2
     L = w.lens()
+    if w.q is not None:
+        # shared latent (K = V = the FP4 latent, 288 B per token): the step is
+        # the decode alone (q in, x out); scores and aggregation both Ckv wide
+        entry = w.Ckv // 2 + w.Ckv // 16
+        HQ = w.H * w.Q
+        vis = float(L.sum())
+        b = vis * entry + w.B * HQ * w.Ckv * es * 2
+        fl = vis * w.Q * w.H * 2 * (2 * w.Ckv)
+        return dict(decode_bytes=b, decode_flops=fl, step_bytes=b, step_flops=fl)
     if w.causal:
         vis_rows = sum(int(l) - w.Q + 1 + q for l in L for q in range(w.Q)) / w.Q
     else:
@@ -261,32 +278,47 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def up(a, dtype=dt):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dtype).to(dev)
 
-    q_nope, q_pe, wkv_b = up(w.q_nope), up(w.q_pe), up(w.wkv_b)
-    if w.block_table is not None:
-        kv, pe = up(w.kv_pool), up(w.pe_pool)
-        bt = torch.from_numpy(w.block_table).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    shared = w.q is not None
+    if shared:
+        # shared-latent variant (FP4 latent, sink, inverse RoPE): the step is
+        # the decode (+ combine); q in, x out
+        from latent_kv_decode_b200 import workloads as wlmod
+        q = up(w.q)
+        kv = torch.from_numpy(wlmod.fp4_random_entries(w.B, w.Lk, w.Ckv)).to(dev)
+        sinks = torch.from_numpy(w.sinks.astype(np.float32)).to(dev)
+        call = ops.make_decode_args(q, None, kv, None, w.softmax_scale, sinks=sinks,
+                                    rope_tail=w.rope_tail, rope_theta=w.rope_theta,
+                                    num_splits=args.num_splits, Lk=w.Lk)
+        h2d = [q]
+        out = call.x
     else:
-        kv, pe = up(w.kv_cache), up(w.pe_cache)
-        bt = None
-    seq_lens = torch.from_numpy(w.seq_lens).to(dev) if w.seq_lens is not None else None
-    B, H, Q = w.B, w.H, w.Q
-    q_lat = torch.empty((B, H, Q, w.Ckv), dtype=dt, device=dev)
-    out = torch.empty((B, H, Q, w.Vd), dtype=dt, device=dev)
-    call = ops.make_decode_args(q_lat, q_pe, kv, pe, w.softmax_scale, seq_lens=seq_lens,
-                                block_table=bt, page_size=w.page_size, causal=w.causal,
-                                num_splits=args.num_splits,
-                                Lk=w.Lk if bt is None else None)
+        q_nope, q_pe, wkv_b = up(w.q_nope), up(w.q_pe), up(w.wkv_b)
+        if w.block_table is not None:
+            kv, pe = up(w.kv_pool), up(w.pe_pool)
+            bt = torch.from_numpy(w.block_table).to(dev)
+        else:
+            kv, pe = up(w.kv_cache), up(w.pe_cache)
+            bt = None
+        seq_lens = torch.from_numpy(w.seq_lens).to(dev) if w.seq_lens is not None else None
+        q_lat = torch.empty((w.B, w.H, w.Q, w.Ckv), dtype=dt, device=dev)
+        out = torch.empty((w.B, w.H, w.Q, w.Vd), dtype=dt, device=dev)
+        call = ops.make_decode_args(q_lat, q_pe, kv, pe, w.softmax_scale, seq_lens=seq_lens,
+                                    block_table=bt, page_size=w.page_size, causal=w.causal,
+                                    num_splits=args.num_splits,
+                                    Lk=w.Lk if bt is None else None)
+        h2d = [q_nope, q_pe]
     need = ops.workspace_bytes(call)
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
     split = call.num_splits > 1
-    launches_per_step = 3 + (1 if split else 0)
+    launches_per_step = (1 if shared else 3) + (1 if split else 0)
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        ops.mla_absorb_q(q_nope, wkv_b, q_lat, stream=stream)
+        if not shared:
+            ops.mla_absorb_q(q_nope, wkv_b, q_lat, stream=stream)
         if evs:
             evs[1].record(stream)
         ops.launch_decode(call, ws, stream=stream)
@@ -296,7 +328,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             ops.mla_combine(call, stream=stream)
         if evs:
             evs[3].record(stream)
-        ops.mla_up_proj(call.x, wkv_b, w.Dn, out, stream=stream)
+        if not shared:
+            ops.mla_up_proj(call.x, wkv_b, w.Dn, out, stream=stream)
         if evs:
             evs[4].record(stream)
 
@@ -340,14 +373,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     up_ms = [e[3].elapsed_time(e[4]) for e in bevs]
     mean_dec = sum(dec_ms) / KB
 
-    # end to end: H2D of this step's queries from pinned memory, the four calls, D2H of out
-    h_qn = q_nope.cpu().pin_memory()
-    h_qp = q_pe.cpu().pin_memory()
-    h_out = torch.empty(out.shape, dtype=dt).pin_memory()
+    # end to end: H2D of this step's queries from pinned memory, the calls, D2H of out
+    h_in = [t.cpu().pin_memory() for t in h2d]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for _ in range(3):
-        q_nope.copy_(h_qn, non_blocking=True)
-        q_pe.copy_(h_qp, non_blocking=True)
+        for d_t, h_t in zip(h2d, h_in):
+            d_t.copy_(h_t, non_blocking=True)
         step()
         h_out.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
@@ -356,8 +388,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for i in range(K):
         flush.fill_(float(i))
         e2e_ev[i][0].record(stream)
-        q_nope.copy_(h_qn, non_blocking=True)
-        q_pe.copy_(h_qp, non_blocking=True)
+        for d_t, h_t in zip(h2d, h_in):
+            d_t.copy_(h_t, non_blocking=True)
         step()
         h_out.copy_(out, non_blocking=True)
         e2e_ev[i][1].record(stream)
@@ -394,17 +426,32 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "data": "synthetic (seeded N(0,1) inputs, wkv_b N(0,1)/sqrt(512), no trained weights)",
         "config": dict(workload_desc(w), parallelism=f"dp{world}" if world > 1 else "single GPU",
                        num_splits=call.num_splits),
-        "roofline": {
-            "kernel": "mla_decode (decode kernel, one launch per step)",
-            "bound": "hbm",
-            "achieved": round(dec_gbs, 1),
-            "peak": hbm,
-            "unit": "GB/s",
-            "frac": round(dec_gbs / hbm, 4),
-            "traffic": profiled_traffic(args.workload),
-            "peak_source": f"hbm_gbs of {psrc}",
-            "algorithmic_bytes_per_launch": int(alg["decode_bytes"]),
-        },
+        "roofline": (
+            {
+                "kernel": "mla_decode (decode kernel, one launch per step)",
+                "bound": "hbm",
+                "achieved": round(dec_gbs, 1),
+                "peak": hbm,
+                "unit": "GB/s",
+                "frac": round(dec_gbs / hbm, 4),
+                "traffic": profiled_traffic(args.workload),
+                "peak_source": f"hbm_gbs of {psrc}",
+                "algorithmic_bytes_per_launch": int(alg["decode_bytes"]),
+            }
+            if alg["decode_bytes"] / (hbm * 1e9) >= alg["decode_flops"] / (tflops * 1e12) else
+            {
+                "kernel": "mla_decode (decode kernel, one launch per step)",
+                "bound": "tensor",
+                "achieved": round(alg["decode_flops"] / (mean_dec * 1e-3) / 1e12, 2),
+                "peak": tflops,
+                "unit": "TFLOP/s",
+                "frac": round(alg["decode_flops"] / (mean_dec * 1e-3) / 1e12 / tflops, 4),
+                "traffic": profiled_traffic(args.workload),
+                "peak_source": f"bf16_tflops of {psrc} (dense bf16 MMA; the FP4 cache is dequantised to bf16)",
+                "algorithmic_flops_per_launch": int(alg["decode_flops"]),
+                "algorithmic_bytes_per_launch": int(alg["decode_bytes"]),
+            }
+        ),
         "step": {
             "bytes": int(alg["step_bytes"]), "flops": int(alg["step_flops"]),
             "TB_per_s": round(step_gbs / 1e3, 4), "TFLOP_per_s": round(step_tf, 2),
@@ -420,11 +467,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "e2e": {
             "value": round(job_tokens_per_s(w.B, w.Q, world, e2e_mean), 1), "unit": "tokens/s",
             "ms_per_step": round(e2e_mean, 5),
-            "h2d_bytes_per_step": int(q_nope.numel() * q_nope.element_size() +
-                                      q_pe.numel() * q_pe.element_size()),
+            "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in h2d)),
             "d2h_bytes_per_step": int(out.numel() * out.element_size()),
-            "path": "pinned host q_nope/q_pe -> mla_absorb_q -> mla_decode -> mla_combine -> "
-                    "mla_up_proj -> pinned host out, one stream",
+            "path": ("pinned host q -> mla_decode -> mla_combine -> pinned host x, one stream"
+                     if shared else
+                     "pinned host q_nope/q_pe -> mla_absorb_q -> mla_decode -> mla_combine -> "
+                     "mla_up_proj -> pinned host out, one stream"),
         },
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),

@@ -247,6 +247,21 @@ def v41_shared_latent(B: int = 32, Lk: int = 8192, H: int = 64, seed: int = 4) -
     return make_shared_latent(B, H, 1, Lk, seed=seed, name=f"v41_fp4_sink_h{H}")
 
 
+def fp4_random_entries(B: int, Lk: int, Ckv: int = 512, seed: int = 5) -> np.ndarray:
+    """(B, Lk, Ckv/2 + Ckv/16) uint8 cache entries for timing: Ckv/2 bytes of
+    uniformly random E2M1 code pairs, then Ckv/16 random E4M3 scale bytes
+    drawn from the finite, non-zero codes (exponent field 1..14). Valid
+    entries with no encoding step; parity tests use the cache-write step's
+    entries instead."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    codes = rng.integers(0, 256, size=(B, Lk, Ckv // 2), dtype=np.uint8)
+    exp = rng.integers(1, 15, size=(B, Lk, Ckv // 16), dtype=np.uint8)
+    mant = rng.integers(0, 8, size=(B, Lk, Ckv // 16), dtype=np.uint8)
+    sign = rng.integers(0, 2, size=(B, Lk, Ckv // 16), dtype=np.uint8)
+    scales = (sign << 7) | (exp << 3) | mant
+    return np.concatenate([codes, scales], axis=-1)
+
+
 WORKLOADS = {
     "demo_fp32": demo_fp32,
     "dsv3_b64_lk4096": dsv3,
