@@ -1,0 +1,623 @@
+// Tensor-core decode for the shared-latent FP4 cache (the openarchlab
+// DeepSeek-V4.1-Flash page, sections on the 288-byte latent entry and the
+// attention sink): K = V = the 512-wide latent, dequantised from E2M1 codes
+// with one E4M3 scale per 16 channels; the softmax denominator takes the sink
+// logit once; x's last 64 dims are rotated back by the query position.
+//
+// One CTA per (64-row query block, sequence, split); 1-SM tcgen05 MMAs with
+// M = 64 (the query block). Per 32-token tile:
+//
+//   load       one bulk copy of the tile's 32 contiguous 288-byte entries
+//   dequant    4 warps decode each entry to 512 bf16 into a tile stored in
+//              the 128-byte-swizzled layout the MMAs read: K-major rows for
+//              S = Q . K^T, and the same bytes as the MN-major V of O += P.V
+//              (one tile serves both, so every entry is read once). Every
+//              E2M1 x E4M3 product is exact in bf16. Rows past the sequence
+//              are stored as zeros.
+//   S = Q.K^T  M = 64, N = 32, K = 512 (32 MMAs of K = 16)
+//   softmax    one lane per row (lanes 0-15 of each TMEM subpartition hold an
+//              M = 64 result), base 2, lazy rescale (threshold 2^8)
+//   O += P.V   2 MMAs of N = 256 per 16 tokens; the first 256 columns of O
+//              sit in lanes 0-15 of each subpartition, the second 256 in
+//              lanes 16-31 (the interleaved M = 64 placement), so O takes
+//              256 TMEM columns and the four S buffers 128 more.
+//
+// Shared memory: Q 64 KB; entry ring 4 x 9 KB; bf16 tile ring 3 x 32 KB;
+// P 2 x 4 KB (64-byte swizzle); decode tables 1.5 KB.
+//
+// Warp roles (320 threads): warp 0 loader (Q, entries), warp 1 MMA issuer and
+// TMEM owner, warps 2-5 dequant, warps 6-9 softmax + epilogue. Every wait is
+// bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kLoaderWarp = 0, kMmaWarp = 1, kDeqWarp0 = 2, kSoftWarp0 = 6;
+constexpr int kTT = 32;                     // tokens per tile
+constexpr int kRows = 64;                   // query rows per CTA
+constexpr int kEntry = 288;                 // bytes per FP4 entry (512 codes + 32 scales)
+constexpr int kRawStages = 4;
+constexpr int kRawStage = kTT * kEntry;     // 9216 B
+constexpr int kKStages = 3;
+constexpr int kKChunk = kTT * 128;          // 32 rows x 64 dims bf16 (4 KB)
+constexpr int kKStage = 8 * kKChunk;        // 32 KB
+constexpr int kPBufs = 2;
+constexpr int kPBuf = kRows * kTT * 2;      // 4 KB, 64-byte rows
+constexpr int kSBufs = 4;
+
+constexpr int kOffQ = 0;
+constexpr int kOffRaw = kOffQ + 8 * 8192;
+constexpr int kOffK = kOffRaw + kRawStages * kRawStage;
+constexpr int kOffP = kOffK + kKStages * kKStage;
+constexpr int kOffLut2 = kOffP + kPBufs * kPBuf;     // 256 x u32: bf16x2 of a code byte's two nibbles
+constexpr int kOffLut1 = kOffLut2 + 1024;            // 256 x u16: bf16 of an E4M3 byte
+constexpr int kOffBar = kOffLut1 + 512;
+enum : int {
+  B_QFULL = 0,
+  B_RAWFULL = B_QFULL + 1,
+  B_RAWEMPTY = B_RAWFULL + kRawStages,
+  B_KFULL = B_RAWEMPTY + kRawStages,
+  B_KEMPTY = B_KFULL + kKStages,
+  B_SFULL = B_KEMPTY + kKStages,
+  B_SFREE = B_SFULL + kSBufs,
+  B_PFULL = B_SFREE + kSBufs,
+  B_PVDONE = B_PFULL + kPBufs,
+  B_COUNT = B_PVDONE + kPBufs
+};
+constexpr int kOffTmemPtr = kOffBar + B_COUNT * 8;
+constexpr int kOffAbort = kOffTmemPtr + 4;
+constexpr int kSmemBytes = kOffBar + 512;
+constexpr int kSmemAlloc = kSmemBytes + 1024;
+static_assert(kOffAbort + 4 <= kSmemBytes, "barrier area overflow");
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kOffRaw % 1024 == 0 && kOffK % 1024 == 0 && kOffP % 1024 == 0, "1 KB swizzle atoms");
+
+constexpr uint32_t kColO = 0;               // O: columns 0-255, lanes 0-15 (dims 0-255) and 16-31 (256-511)
+constexpr uint32_t kColS = 256;             // S buffer i at columns 256 + 32 i, lanes 0-15
+constexpr uint32_t kTmemCols = 512;
+
+constexpr float kRescaleThreshold = 8.0f;
+static_assert(kTT == 32, "visibility is one 32-bit mask per tile");
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct alignas(64) Fp4Params {
+  CUtensorMap tm_q;   // q (B*HQ, 512) bf16, box 64 x 64
+  DecodeParams p;
+  int paged;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Page table entry of token t is usable (paged caches only).
+__device__ __forceinline__ bool page_ok(const DecodeParams& p, int b, int t) {
+  if (!p.block_table) return true;
+  const int pg = p.block_table[(int64_t)b * p.max_pages + (t >> 6)];
+  return pg >= 0 && pg < p.num_pages;
+}
+
+__device__ __forceinline__ uint32_t swz128(int r, int u) {
+  return (uint32_t)r * 128u + ((uint32_t)((u & 7) ^ (r & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __grid_constant__ Fp4Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb0 = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sb0 - raw);
+  const DecodeParams& p = P.p;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rb = blockIdx.x, b = blockIdx.y, z = blockIdx.z;
+  auto bar = [&](int i) -> uint32_t { return sb0 + kOffBar + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  pdl_launch_dependents();
+
+  // decode tables (exact: E2M1 and E4M3 values are bf16 values)
+  {
+    uint32_t* lut2 = reinterpret_cast<uint32_t*>(smem + kOffLut2);
+    uint16_t* lut1 = reinterpret_cast<uint16_t*>(smem + kOffLut1);
+    for (int i = threadIdx.x; i < 256; i += kThreads) {
+      lut2[i] = pack_bf16(e2m1_value((uint32_t)i & 15u), e2m1_value((uint32_t)i >> 4));
+      lut1[i] = __bfloat16_as_ushort(__float2bfloat16_rn(e4m3_value((uint32_t)i)));
+    }
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < kRawStages; ++s) {
+      mbar_init(bar(B_RAWFULL + s), 1);
+      mbar_init(bar(B_RAWEMPTY + s), 4);   // one arrival per dequant warp
+    }
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(B_KFULL + s), 4);      // one arrival per dequant warp
+      mbar_init(bar(B_KEMPTY + s), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(bar(B_SFULL + i), 1);
+      mbar_init(bar(B_SFREE + i), 1);
+    }
+    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(bar(B_PFULL + i), 1);
+      mbar_init(bar(B_PVDONE + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sb0 + kOffTmemPtr, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemPtr);
+  // everything above overlapped the previous kernel; global inputs are read
+  // only once that grid has completed
+  pdl_wait();
+  const int len = seq_len_of(p, b);
+  int t_begin, t_end;
+  split_range(len, p.num_splits, z, t_begin, t_end);
+  const int ntiles = (t_end - t_begin + kTT - 1) / kTT;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    flag_error(p, MLA_DEVICE_ERR_TIMEOUT);
+  };
+  const uint8_t* kvb = reinterpret_cast<const uint8_t*>(p.kv);
+
+  if (warp == kLoaderWarp) {
+    // ------------------------------------------------------------------ loader
+    if (lane == 0) {
+      tma_prefetch_desc(&P.tm_q);
+      const int qrow = b * p.HQ + rb * kRows;
+      mbar_arrive_expect_tx(bar(B_QFULL), 8 * 8192);
+      for (int c = 0; c < 8; ++c) tma_load_2d(sb0 + kOffQ + c * 8192, &P.tm_q, bar(B_QFULL), 64 * c, qrow);
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int s = j % kRawStages;
+        if (j >= kRawStages && !mbar_wait(bar(B_RAWEMPTY + s), ((j / kRawStages) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const int t0 = t_begin + j * kTT;
+        const uint8_t* src;
+        int n = kTT;
+        if (P.paged) {
+          int pg = 0;
+          if (t0 < len) {
+            pg = p.block_table[(int64_t)b * p.max_pages + (t0 >> 6)];
+            if (pg < 0 || pg >= p.num_pages) {
+              flag_error(p, MLA_DEVICE_ERR_BLOCK_TABLE);
+              pg = 0;   // its tokens are masked by the softmax
+            }
+          }
+          src = kvb + ((int64_t)pg * 64 + (t0 & 63)) * kEntry;
+        } else {
+          src = kvb + (int64_t)b * p.kv_batch + (int64_t)t0 * kEntry;
+          n = min(kTT, p.Lk - t0);   // stay inside this sequence's rows
+        }
+        mbar_arrive_expect_tx(bar(B_RAWFULL + s), (uint32_t)(n * kEntry));
+        bulk_load(sb0 + kOffRaw + s * kRawStage, src, (uint32_t)(n * kEntry), bar(B_RAWFULL + s));
+        if (*abort_flag) ok = false;
+      }
+      if (!ok) fail();
+    }
+    __syncwarp();
+  } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + 4) {
+    // ------------------------------------------------------------------ dequant
+    // 2048 pieces of 8 channels per tile, 16 per thread: piece i = token
+    // i/64, chunk (i/8)%8, 16-byte unit i%8 (channels 64 chunk + 8 unit)
+    const int dt = threadIdx.x - kDeqWarp0 * 32;   // 0..127
+    const uint32_t* lut2 = reinterpret_cast<const uint32_t*>(smem + kOffLut2);
+    const uint16_t* lut1 = reinterpret_cast<const uint16_t*>(smem + kOffLut1);
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int rs = j % kRawStages, ks = j % kKStages;
+      bool got = mbar_wait(bar(B_RAWFULL + rs), (j / kRawStages) & 1);
+      if (got && j >= kKStages) got = mbar_wait(bar(B_KEMPTY + ks), ((j / kKStages) - 1) & 1);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* rawp = smem + kOffRaw + rs * kRawStage;
+      const uint32_t kbase = sb0 + kOffK + ks * kKStage;
+      const int t0 = t_begin + j * kTT;
+#pragma unroll 4
+      for (int k = 0; k < 16; ++k) {
+        const int i = dt + 128 * k, t = i >> 6, c = (i >> 3) & 7, u = i & 7;
+        uint4 out = make_uint4(0, 0, 0, 0);
+        if (t0 + t < len) {
+          const uint8_t* e = rawp + t * kEntry;
+          const uint32_t codes = *reinterpret_cast<const uint32_t*>(e + 32 * c + 4 * u);
+          const uint32_t sc = lut1[e[256 + 4 * c + (u >> 1)]];
+          const __nv_bfloat162 s2 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)sc),
+                                                       __ushort_as_bfloat16((unsigned short)sc));
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t pr = lut2[(codes >> (8 * q)) & 0xffu];
+            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pr);
+            const __nv_bfloat162 m = __hmul2(v, s2);
+            w[q] = *reinterpret_cast<const uint32_t*>(&m);
+          }
+          out = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *reinterpret_cast<uint4*>(smem + (kbase - sb0) + c * kKChunk + swz128(t, u)) = out;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(B_KFULL + ks));
+        mbar_arrive(bar(B_RAWEMPTY + rs));
+      }
+      if (*abort_flag) ok = false;
+      ok = __all_sync(0xffffffffu, ok) != 0;
+    }
+    if (!ok && lane == 0) fail();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(kRows, kTT, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);
+      bool ok = mbar_wait(bar(B_QFULL), 0);
+      int qj = 0, pj = 0;
+      uint64_t t_idle = global_ns();
+      uint32_t idle = 0;
+      while (ok && pj < ntiles) {
+        bool prog = false;
+        if (qj < ntiles) {
+          const int sbuf = qj % kSBufs, ks = qj % kKStages;
+          const bool sfree = qj < kSBufs || mbar_poll(bar(B_SFREE + sbuf), ((qj / kSBufs) - 1) & 1);
+          if (sfree && mbar_poll(bar(B_KFULL + ks), (qj / kKStages) & 1)) {
+            tc_fence_after();
+            const uint32_t kb = sb0 + kOffK + ks * kKStage;
+#pragma unroll 4
+            for (int kk = 0; kk < 32; ++kk) {
+              const int c = kk >> 2, sub = kk & 3;
+              mma_bf16_ss(tmem + kColS + 32u * sbuf,
+                          smem_desc(sb0 + kOffQ + c * 8192 + 32 * sub, 16, 1024, kSwizzle128B),
+                          smem_desc(kb + c * kKChunk + 32 * sub, 16, 1024, kSwizzle128B), idesc_qk,
+                          kk > 0);
+            }
+            mma_commit(bar(B_SFULL + sbuf));
+            ++qj;
+            prog = true;
+          }
+        }
+        if (pj < qj) {
+          const int pb = pj % kPBufs, ks = pj % kKStages;
+          if (mbar_poll(bar(B_PFULL + pb), (pj / kPBufs) & 1)) {
+            tc_fence_after();
+            const uint32_t kb = sb0 + kOffK + ks * kKStage;
+            const uint32_t pa = sb0 + kOffP + pb * kPBuf;
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {
+                // P: 16 tokens per step (K-major, 64-byte rows); V: the tile's
+                // chunks 4n..4n+3 (MN-major); D: lanes 16n.. of each subpartition
+                mma_bf16_ss(tmem + ((16u * n) << 16) + kColO,
+                            smem_desc(pa + 32 * kk, 16, 512, kSwizzle64B),
+                            smem_desc(kb + 4 * n * kKChunk + 2048 * kk, kKChunk, 1024, kSwizzle128B),
+                            idesc_pv, (pj > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit(bar(B_KEMPTY + ks));
+            mma_commit(bar(B_PVDONE + pb));
+            ++pj;
+            prog = true;
+          }
+        }
+        if (prog) {
+          idle = 0;
+        } else {
+          // nothing ready: yield the issue slots this sub-partition shares
+          // with a dequant and a softmax warp
+          __nanosleep(64);
+          if ((++idle & 255u) == 0) {
+            if (idle == 256u) t_idle = global_ns();
+            else if (global_ns() - t_idle > 1000000000ull || *abort_flag) ok = false;
+          }
+        }
+      }
+      if (!ok) fail();
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    // Warp g = warp % 4 owns TMEM subpartition g: lane i < 16 holds row
+    // 16 g + i of S and the first 256 columns of its O row; lane 16 + i holds
+    // the second 256 columns of the same row.
+    const int g = warp & 3;
+    const int hi = lane >> 4, m = 16 * g + (lane & 15);
+    const int r = rb * kRows + m;
+    const int q = r % p.Q;
+    const int h = r / p.Q;
+    const uint32_t lane_base = (uint32_t)(32 * g) << 16;
+    const float sl2 = p.scale_log2;
+    const uint8_t* mask = p.mask;
+    const bool causal = p.causal != 0;
+    const int causal_last = len - p.Q + q;
+    const bool paged = p.block_table != nullptr;
+    const bool leader = (warp == kSoftWarp0 && lane == 0);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ab = false;
+    auto wait_pv = [&](int t) {
+      if (!ab) ab = !mbar_wait(bar(B_PVDONE + (t % kPBufs)), (t / kPBufs) & 1);
+    };
+    for (int j = 0; j < ntiles; ++j) {
+      const int sbuf = j % kSBufs, pb = j % kPBufs;
+      if (!ab) ab = !mbar_wait(bar(B_SFULL + sbuf), (j / kSBufs) & 1);
+      ab = __any_sync(0xffffffffu, ab);
+      float s[kTT];
+      if (!ab) {
+        tc_fence_after();
+        uint32_t v[2][16];
+        tmem_ld16(tmem + lane_base + kColS + 32u * sbuf, v[0]);
+        tmem_ld16(tmem + lane_base + kColS + 32u * sbuf + 16u, v[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          s[i] = __uint_as_float(v[0][i]);
+          s[16 + i] = __uint_as_float(v[1][i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTT; ++i) s[i] = 0.f;
+      }
+      tc_fence_before();
+      named_bar_sync(1, 128);   // every warp has read S(j)
+      if (leader) mbar_arrive(bar(B_SFREE + sbuf));
+
+      const int tb = t_begin + j * kTT;
+      int lim = t_end - tb;
+      if (causal) lim = min(lim, causal_last - tb + 1);
+      if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;
+      if (ab) lim = 0;
+      // visibility of the tile's 32 tokens as a bit mask: the question's mask
+      // is read once per token, one lane each (tb is the same for every row)
+      uint32_t vbits = lim >= kTT ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+      if (mask != nullptr) vbits &= __ballot_sync(0xffffffffu, tb + lane < t_end && mask[tb + lane] != 0);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTT; ++c) {
+        s[c] = ((vbits >> c) & 1u) ? s[c] * sl2 : -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = (m_new - m_run) > kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = exp2f(m_run - m_new);
+        m_run = m_new;
+      }
+      uint32_t pk[kTT / 2];
+      float psum = 0.f;
+      const bool none = (m_run == -INFINITY);
+#pragma unroll
+      for (int c = 0; c < kTT / 2; ++c) {
+        const float p0 = none ? 0.f : fast_exp2(s[2 * c] - m_run);
+        const float p1 = none ? 0.f : fast_exp2(s[2 * c + 1] - m_run);
+        psum += p0 + p1;
+        pk[c] = pack_bf16(p0, p1);
+      }
+      l_run = l_run * alpha + psum;
+      // lanes 16-31 rescale the second half of the same rows: take lane i's alpha
+      const float alpha_row = __shfl_sync(0xffffffffu, alpha, lane & 15);
+      const bool need_row = __shfl_sync(0xffffffffu, need, lane & 15);
+
+      if (j >= kPBufs) wait_pv(j - kPBufs);
+      if (hi == 0) {
+        uint8_t* prow = smem + kOffP + pb * kPBuf + m * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + 16 * (c ^ ((m >> 1) & 3))) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      if (__any_sync(0xffffffffu, need_row && j > 0)) {
+        wait_pv(j - 1);
+        ab = __any_sync(0xffffffffu, ab);
+        if (!ab) {
+          tc_fence_after();
+          // 256 columns in 4 rounds of 64: four loads per wait
+#pragma unroll 1
+          for (int c = 0; c < 16; c += 4) {
+            uint32_t v[4][16];
+            const uint32_t ta = tmem + lane_base + kColO + 16u * c;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tmem_ld16(ta + 16u * k, v[k]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[k][i] = __float_as_uint(__uint_as_float(v[k][i]) * alpha_row);
+              tmem_st16(ta + 16u * k, v[k]);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(1, 128);   // P(j) of every row is written
+      if (leader) mbar_arrive(bar(B_PFULL + pb));
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ntiles > 0) wait_pv(ntiles - 1);
+    ab = __any_sync(0xffffffffu, ab);
+    if (ab && lane == 0) fail();
+    tc_fence_after();
+    const bool have_o = ntiles > 0 && !ab;
+    const float mrow = __shfl_sync(0xffffffffu, m_run, lane & 15);
+    const float lrow = __shfl_sync(0xffffffffu, l_run, lane & 15);
+    const int64_t grow = (int64_t)b * p.HQ + r;
+    float scale_o, lse;
+    if (p.num_splits > 1) {
+      scale_o = lrow > 0.f ? 1.f / lrow : 0.f;
+      lse = lrow > 0.f ? (mrow + log2f(lrow)) * kLn2 : -INFINITY;
+    } else {
+      float mfin = mrow, lfin = lrow, w = 1.f;
+      if (p.sinks) {
+        const float sk = p.sinks[h] * kLog2e;
+        const float m2 = fmaxf(mrow, sk);
+        w = (mrow == -INFINITY) ? 0.f : exp2f(mrow - m2);
+        lfin = lrow * w + exp2f(sk - m2);
+        mfin = m2;
+      }
+      scale_o = lfin > 0.f ? w / lfin : 0.f;
+      lse = lfin > 0.f ? (mfin + log2f(lfin)) * kLn2 : -INFINITY;
+    }
+#pragma unroll 1
+    for (int c = 0; c < 16; ++c) {
+      uint32_t v[16];
+      if (have_o) {
+        tmem_ld16(tmem + lane_base + kColO + 16u * c, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0u;
+      }
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * scale_o;
+      const int col = 256 * hi + 16 * c;
+      if (p.num_splits > 1) {
+        float* o = p.ws_o + ((int64_t)z * p.B * p.HQ + grow) * p.Ckv + col;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(o + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+      } else {
+        if (p.rope_tail > 0 && col >= p.Ckv - p.rope_tail) {
+          const int pos = len - p.Q + q;
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const int jp = (col + i - (p.Ckv - p.rope_tail)) >> 1;
+            inverse_rope_pair(f[i], f[i + 1], jp, p.rope_tail, p.rope_theta, pos);
+          }
+        }
+        uint32_t w4[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w4[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.x) + grow * p.Ckv + col);
+        o[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        o[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+      }
+    }
+    if (hi == 0) {
+      if (p.num_splits > 1)
+        p.ws_lse[(int64_t)z * p.B * p.HQ + grow] = lse;
+      else if (p.lse)
+        p.lse[grow] = lse;
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 fp4_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool sm100_fp4_decode_supported(const mla_decode_args* a) {
+  if (a->cache_dtype != MLA_FP4_E2M1_E4M3x16 || a->q_dtype != MLA_BF16) return false;
+  if (a->Ckv != 512 || a->Dr != 0) return false;
+  if ((a->H * a->Q) % kRows != 0) return false;
+  if (a->kv_row_stride != kEntry) return false;            // contiguous entries: one bulk copy per tile
+  if (a->block_table) {
+    if (a->page_size != 64) return false;
+  } else if (a->kv_batch_stride % 16 != 0) {
+    return false;
+  }
+  if ((reinterpret_cast<uintptr_t>(a->q_lat) & 15u) || (reinterpret_cast<uintptr_t>(a->kv_cache) & 15u))
+    return false;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10 && fp4_encode_fn() != nullptr;
+}
+
+int sm100_fp4_auto_splits(const mla_decode_args* a, int sms) {
+  const int ctas = a->B * (a->H * a->Q / kRows);
+  const int tiles = (a->Lk + kTile - 1) / kTile;
+  if (ctas >= sms) return 1;
+  int s = sms / ctas;
+  if (s > tiles) s = tiles;
+  return s < 1 ? 1 : s;
+}
+
+cudaError_t launch_decode_fp4_sm100(const DecodeParams& p, const mla_decode_args* a, cudaStream_t st) {
+  Fp4Params P;
+  memset(&P, 0, sizeof(P));
+  P.p = p;
+  P.paged = a->block_table != nullptr;
+  {
+    auto fn = fp4_encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    cuuint64_t d[2] = {512, (cuuint64_t)p.B * p.HQ};
+    cuuint64_t s[1] = {512 * 2};
+    cuuint32_t box[2] = {64, 64}, es[2] = {1, 1};
+    if (fn(&P.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a->q_lat), d, s, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(decode_fp4_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.HQ / kRows, p.B, p.num_splits);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_fp4_sm100_kernel, P);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -148,10 +148,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   const uint32_t rank = cluster_ctarank();
   const int rb = blockIdx.x >> 1, b = blockIdx.y, z = blockIdx.z;
   pdl_launch_dependents();
-  const int len = seq_len_of(p, b);
-  int t_begin, t_end;
-  split_range(len, p.num_splits, z, t_begin, t_end);
-  const int ntiles = (t_end - t_begin + kTileT - 1) / kTileT;
   auto bar = [&](int i) -> uint32_t { return sb0 + kOffBar + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
@@ -182,6 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemPtr);
+  // the setup above overlapped the previous kernel (the absorb); global
+  // inputs (q_lat, lengths, tables, the cache) are read only once it completed
+  pdl_wait();
+  const int len = seq_len_of(p, b);
+  int t_begin, t_end;
+  split_range(len, p.num_splits, z, t_begin, t_end);
+  const int ntiles = (t_end - t_begin + kTileT - 1) / kTileT;
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -203,9 +206,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       tma_prefetch_desc(&P.tm_k);
       tma_prefetch_desc(&P.tm_k3);
       tma_prefetch_desc(&P.tm_pe);
-      // q_lat comes from the previous kernel (the absorb): read it only once
-      // that grid has completed; everything above overlapped its tail
-      pdl_wait();
       const int qrow = b * p.HQ + rb * 128 + (int)rank * 64;
       const uint32_t qbar = map_to_rank(bar(B_QFULL), 0);
       if (rank == 0) mbar_arrive_expect_tx(bar(B_QFULL), 2 * kQBytes);
@@ -428,9 +428,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
           mx = fmaxf(mx, s[c]);
         }
       } else {
+        // the question's mask, one byte per lane (tb is the same across the warp)
+        const uint32_t m0 = __ballot_sync(0xffffffffu, tb + lane < t_end && mask[tb + lane] != 0);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, tb + 32 + lane < t_end && mask[tb + 32 + lane] != 0);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const bool vis = c < lim && mask[tb + c] != 0;
+          const bool vis = c < lim && (((c < 32 ? m0 : m1) >> (c & 31)) & 1u);
           s[c] = vis ? s[c] * sl2 : -INFINITY;
           mx = fmaxf(mx, s[c]);
         }
@@ -477,15 +480,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         ab = __any_sync(0xffffffffu, ab);
         if (!ab) {
           tc_fence_after();
+          // 256 columns in 4 rounds of 64: four loads per wait
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
-            uint32_t v[16];
+          for (int c = 0; c < 16; c += 4) {
+            uint32_t v[4][16];
             const uint32_t ta = tmem + lane_base + kColO + 16u * c;
-            tmem_ld16(ta, v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tmem_ld16(ta + 16u * k, v[k]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st16(ta, v);
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[k][i] = __float_as_uint(__uint_as_float(v[k][i]) * alpha);
+              tmem_st16(ta + 16u * k, v[k]);
+            }
           }
           tmem_wait_st();
         }

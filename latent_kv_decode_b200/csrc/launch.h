@@ -24,6 +24,12 @@ cudaError_t launch_absorb_sm100(const void* q_nope, const void* wkv_b, void* q_l
 cudaError_t launch_up_proj_sm100(const void* x, const void* wkv_b, void* out, int B, int H, int Q,
                                  int Dn, int Vd, int Ckv, cudaStream_t st);
 
+// tensor-core (tcgen05, 1-SM, M = 64) decode for the shared-latent FP4 cache: bf16 q,
+// Ckv = 512, Dr = 0, H*Q % 64 == 0, contiguous 288-byte entries (row stride 288)
+bool sm100_fp4_decode_supported(const mla_decode_args* a);
+int sm100_fp4_auto_splits(const mla_decode_args* a, int sms);
+cudaError_t launch_decode_fp4_sm100(const DecodeParams& p, const mla_decode_args* a, cudaStream_t st);
+
 // tensor-core (tcgen05, 2-CTA cluster) decode for bf16, Ckv=512, Dr=64, H*Q % 128 == 0
 bool sm100_decode_supported(const mla_decode_args* a);
 int sm100_auto_splits(const mla_decode_args* a, int sms);

@@ -50,9 +50,11 @@ mla_status_t check_proj(const void* a, const void* w, const void* o, int B, int 
 }
 
 // Which kernel family serves a decode call.
-enum class DecodePath { kSimt, kSm100 };
+enum class DecodePath { kSimt, kSm100, kSm100Fp4 };
 
 DecodePath pick_path(const mla_decode_args* a) {
+  if (a->cache_dtype == MLA_FP4_E2M1_E4M3x16)
+    return mla::sm100_fp4_decode_supported(a) ? DecodePath::kSm100Fp4 : DecodePath::kSimt;
   return mla::sm100_decode_supported(a) ? DecodePath::kSm100 : DecodePath::kSimt;
 }
 
@@ -106,6 +108,7 @@ int resolve_splits(const mla_decode_args* a) {
   if (a->num_splits > 0) return a->num_splits;
   const int tiles = (a->Lk + mla::kTile - 1) / mla::kTile;
   if (pick_path(a) == DecodePath::kSm100) return mla::sm100_auto_splits(a, sm_count());
+  if (pick_path(a) == DecodePath::kSm100Fp4) return mla::sm100_fp4_auto_splits(a, sm_count());
   // generic path: about two CTAs of 16 rows per SM
   const int ctas = a->B * ((a->H * a->Q + 15) / 16);
   int s = (2 * sm_count() + ctas - 1) / ctas;
@@ -229,7 +232,9 @@ mla_status_t mla_decode(const mla_decode_args* a, void* workspace, size_t worksp
     return MLA_ERR_WORKSPACE;
   mla::DecodeParams p = make_params(a, S, workspace);
   cudaStream_t st = (cudaStream_t)stream;
-  if (pick_path(a) == DecodePath::kSm100) return cuda_status(mla::launch_decode_sm100(p, a, st));
+  const DecodePath path = pick_path(a);
+  if (path == DecodePath::kSm100) return cuda_status(mla::launch_decode_sm100(p, a, st));
+  if (path == DecodePath::kSm100Fp4) return cuda_status(mla::launch_decode_fp4_sm100(p, a, st));
   return cuda_status(mla::launch_decode_simt(p, a->q_dtype == MLA_BF16,
                                              a->cache_dtype == MLA_FP4_E2M1_E4M3x16, st));
 }

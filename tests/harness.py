@@ -158,6 +158,7 @@ def gpu_shared_latent(w: wl.Workload, entries: np.ndarray, num_splits: int = 0, 
     call = ops.mla_decode(q, None, kv, None, w.softmax_scale,
                           seq_lens=dev(w.seq_lens) if w.seq_lens is not None else None,
                           block_table=bt, page_size=w.page_size, causal=w.causal, sinks=sinks,
+                          causal_mask=dev(w.causal_mask) if w.causal_mask is not None else None,
                           rope_tail=w.rope_tail, rope_theta=w.rope_theta, num_splits=num_splits,
                           Lk=w.Lk if bt is None else None, err_flag=err_flag)
     ops.mla_combine(call)
@@ -171,5 +172,6 @@ def oracle_shared_latent(w: wl.Workload, entries: np.ndarray, batch=None):
     sel = slice(None) if batch is None else np.asarray(batch)
     r = ov41.shared_latent_decode(w.q[sel], entries[sel], w.sinks, w.softmax_scale,
                                   None if w.seq_lens is None else w.seq_lens[sel], w.causal,
-                                  tail=w.rope_tail, theta=w.rope_theta, return_all=True)
+                                  causal_mask=w.causal_mask, tail=w.rope_tail,
+                                  theta=w.rope_theta, return_all=True)
     return dict(x=r["x"], lse=r["lse"])

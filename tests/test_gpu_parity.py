@@ -135,6 +135,34 @@ def test_shared_latent_fp4_small(splits):
     assert_close(g["lse"], ref["lse"], TOL_BF16, "lse")
 
 
+def test_shared_latent_fp4_causal_q2():
+    """Q = 2 causal rows (row = head * Q + query): 32 heads x 2 queries fill one
+    64-row block; ragged lengths end mid-tile."""
+    w = wl.make_shared_latent(2, 32, 2, 150, seed=23, seq_lens=[150, 97], causal=True)
+    ent = fp4_entries(w)
+    g = gpu_shared_latent(w, ent, num_splits=2)
+    ref = oracle_shared_latent(w, ent)
+    assert_close(g["x"], ref["x"], TOL_BF16, "x", REL_L2_BF16)
+    assert_close(g["lse"], ref["lse"], TOL_BF16, "lse")
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_shared_latent_fp4_question_mask(splits):
+    """The question's (Lk) mask on top of causal Q = 2 rows and ragged lengths:
+    hidden tokens sit inside tiles, at tile edges and in whole 32-token runs."""
+    w = wl.make_shared_latent(2, 32, 2, 200, seed=24, seq_lens=[200, 131], causal=True)
+    rng = np.random.Generator(np.random.PCG64(24))
+    mask = (rng.random(200) > 0.3).astype(np.uint8)
+    mask[[0, 31, 32, 63, 64]] = 0
+    mask[96:128] = 0
+    w.causal_mask = mask
+    ent = fp4_entries(w)
+    g = gpu_shared_latent(w, ent, num_splits=splits)
+    ref = oracle_shared_latent(w, ent)
+    assert_close(g["x"], ref["x"], TOL_BF16, "x", REL_L2_BF16)
+    assert_close(g["lse"], ref["lse"], TOL_BF16, "lse")
+
+
 def test_shared_latent_fp4_paged():
     w = wl.make_shared_latent(3, 64, 1, 260, seed=22, seq_lens=[260, 65, 3], paged=True)
     ent = fp4_entries(w)
