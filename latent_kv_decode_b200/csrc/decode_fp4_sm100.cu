@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kRows, kTT, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);
+      const uint64_t qd = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
       bool ok = mbar_wait(bar(B_QFULL), 0);
       int qj = 0, pj = 0;
       uint64_t t_idle = global_ns();
@@ -294,14 +295,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
           const bool sfree = qj < kSBufs || mbar_poll(bar(B_SFREE + sbuf), ((qj / kSBufs) - 1) & 1);
           if (sfree && mbar_poll(bar(B_KFULL + ks), (qj / kKStages) & 1)) {
             tc_fence_after();
-            const uint32_t kb = sb0 + kOffK + ks * kKStage;
-#pragma unroll 4
+            const uint64_t kd = smem_desc(sb0 + kOffK + ks * kKStage, 16, 1024, kSwizzle128B);
+            const uint32_t d = tmem + kColS + 32u * sbuf;
+#pragma unroll
             for (int kk = 0; kk < 32; ++kk) {
               const int c = kk >> 2, sub = kk & 3;
-              mma_bf16_ss(tmem + kColS + 32u * sbuf,
-                          smem_desc(sb0 + kOffQ + c * 8192 + 32 * sub, 16, 1024, kSwizzle128B),
-                          smem_desc(kb + c * kKChunk + 32 * sub, 16, 1024, kSwizzle128B), idesc_qk,
-                          kk > 0);
+              mma_bf16_ss(d, desc_advance(qd, c * 8192 + 32 * sub),
+                          desc_advance(kd, c * kKChunk + 32 * sub), idesc_qk, kk > 0);
             }
             mma_commit(bar(B_SFULL + sbuf));
             ++qj;
@@ -312,18 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
           const int pb = pj % kPBufs, ks = pj % kKStages;
           if (mbar_poll(bar(B_PFULL + pb), (pj / kPBufs) & 1)) {
             tc_fence_after();
-            const uint32_t kb = sb0 + kOffK + ks * kKStage;
-            const uint32_t pa = sb0 + kOffP + pb * kPBuf;
+            const uint64_t vd = smem_desc(sb0 + kOffK + ks * kKStage, kKChunk, 1024, kSwizzle128B);
+            const uint64_t pd = smem_desc(sb0 + kOffP + pb * kPBuf, 16, 512, kSwizzle64B);
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk) {
                 // P: 16 tokens per step (K-major, 64-byte rows); V: the tile's
                 // chunks 4n..4n+3 (MN-major); D: lanes 16n.. of each subpartition
-                mma_bf16_ss(tmem + ((16u * n) << 16) + kColO,
-                            smem_desc(pa + 32 * kk, 16, 512, kSwizzle64B),
-                            smem_desc(kb + 4 * n * kKChunk + 2048 * kk, kKChunk, 1024, kSwizzle128B),
-                            idesc_pv, (pj > 0 || kk > 0) ? 1u : 0u);
+                mma_bf16_ss(tmem + ((16u * n) << 16) + kColO, desc_advance(pd, 32 * kk),
+                            desc_advance(vd, 4 * n * kKChunk + 2048 * kk), idesc_pv,
+                            (pj > 0 || kk > 0) ? 1u : 0u);
               }
             }
             mma_commit(bar(B_KEMPTY + ks));

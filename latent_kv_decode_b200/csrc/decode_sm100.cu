@@ -303,6 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint64_t qd0 = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
+      const uint64_t kd0 = smem_desc(sb0 + kOffK, 16, 1024, kSwizzle128B);
+      const uint64_t pd0 = smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
+      const uint64_t vd0 = smem_desc(sb0 + kOffV, 8192, 1024, kSwizzle128B);
       bool ok = mbar_wait_cluster(bar(B_QFULL), 0);
       uint32_t kit = 0, vit = 0;
       int qj = 0, qu = 0;   // next QK: tile, stage use (4 latent pairs + rope)
@@ -318,15 +322,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
           if (sfree && mbar_poll_cluster(bar(B_KFULL + s), (kit / kKStages) & 1)) {
             tc_fence_after();
             const uint32_t d = tmem + kColS + 64u * sbuf;
-            const uint32_t kb = sb0 + kOffK + s * kKStage;
+            // Q's 64-dim blocks 3 qu .. 3 qu + 2 (block 8 = rope) against the stage's three
+            const uint64_t qd = desc_advance(qd0, 3 * qu * 8192);
+            const uint64_t kd = desc_advance(kd0, s * kKStage);
+#pragma unroll
             for (int cc = 0; cc < 3; ++cc) {
-              const int c = 3 * qu + cc;                  // 64-dim block of Q (8 = rope)
-              const uint32_t qa = sb0 + kOffQ + c * 8192, ka = kb + cc * 8192;
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                mma_bf16_ss_2sm(d, smem_desc(qa + 32 * k, 16, 1024, kSwizzle128B),
-                                smem_desc(ka + 32 * k, 16, 1024, kSwizzle128B), idesc_qk,
-                                (qu | cc | k) != 0);
+                mma_bf16_ss_2sm(d, desc_advance(qd, cc * 8192 + 32 * k), desc_advance(kd, cc * 8192 + 32 * k),
+                                idesc_qk, (qu | cc | k) != 0);
               }
             }
             mma_commit_2sm_mc(bar(B_KEMPTY + s), 3);
@@ -345,14 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
           if (pready && mbar_poll_cluster(bar(B_VFULL + s), (vit / kVStages) & 1)) {
             tc_fence_after();
             const int n = pu >> 1, th = pu & 1;
-            const uint32_t vb = sb0 + kOffV + s * kStage;
+            const uint64_t pd = desc_advance(pd0, th * 8192);
+            const uint64_t vd = desc_advance(vd0, s * kStage);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               // P: K-block th (64 tokens), 16 tokens per step; V: 2 blocks of 64 columns
-              const uint32_t a_addr = sb0 + kOffP + th * 8192 + 32 * k;
-              mma_bf16_ss_2sm(tmem + kColO + 128u * n, smem_desc(a_addr, 16, 1024, kSwizzle128B),
-                              smem_desc(vb + 2048 * k, 8192, 1024, kSwizzle128B), idesc_pv,
-                              (pj > 0 || th > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_ss_2sm(tmem + kColO + 128u * n, desc_advance(pd, 32 * k), desc_advance(vd, 2048 * k),
+                              idesc_pv, (pj > 0 || th > 0 || k > 0) ? 1u : 0u);
             }
             mma_commit_2sm_mc(bar(B_VEMPTY + s), 3);
             ++vit;

@@ -374,6 +374,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// The same descriptor for an operand `bytes` further on (a multiple of 16).
+// Shared addresses stay below 256 KB, so the 14-bit address field takes the
+// add without carrying into the offsets: two instructions instead of a rebuild.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D:
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   bit 15 A major (0 = K-major, 1 = MN-major), bit 16 B major, bits 17-22 N >> 3,
