@@ -5,31 +5,36 @@
 // logit once; x's last 64 dims are rotated back by the query position.
 //
 // One CTA per (64-row query block, sequence, split); 1-SM tcgen05 MMAs with
-// M = 64 (the query block). Per 32-token tile:
+// M = 64 (the query block). Per 64-token tile:
 //
-//   load       one bulk copy of the tile's 32 contiguous 288-byte entries
-//   dequant    4 warps decode each entry to 512 bf16 into a tile stored in
-//              the 128-byte-swizzled layout the MMAs read: K-major rows for
-//              S = Q . K^T, and the same bytes as the MN-major V of O += P.V
-//              (one tile serves both, so every entry is read once). Every
-//              E2M1 x E4M3 product is exact in bf16. Rows past the sequence
-//              are stored as zeros.
-//   S = Q.K^T  M = 64, N = 32, K = 512 (32 MMAs of K = 16)
+//   load       two bulk copies of 32 contiguous 288-byte entries (a page of
+//              64 tokens holds both halves), plus L2 prefetches two tiles ahead
+//   dequant    8 warps decode each entry to 512 bf16 with byte permutes (no
+//              tables) into a tile stored in the 128-byte-swizzled layout the
+//              MMAs read: K-major rows for S = Q . K^T, and the same bytes as
+//              the MN-major V of O += P.V (one tile serves both, so every entry
+//              is read once). Every E2M1 x E4M3 product is exact in bf16. Rows
+//              past the sequence are stored as zeros.
+//   S = Q.K^T  M = 64, N = 64, K = 512 (32 MMAs of K = 16). An MMA costs about
+//              the same at N = 32 and N = 64, so the wider tile halves the
+//              tensor-pipe time per token of this step.
 //   softmax    one lane per row (lanes 0-15 of each TMEM subpartition hold an
 //              M = 64 result), base 2, lazy rescale (threshold 2^8)
 //   O += P.V   2 MMAs of N = 256 per 16 tokens; the first 256 columns of O
 //              sit in lanes 0-15 of each subpartition, the second 256 in
 //              lanes 16-31 (the interleaved M = 64 placement), so O takes
-//              256 TMEM columns and the four S buffers 128 more.
+//              256 TMEM columns and the two S buffers 128 more.
 //
-// Shared memory: Q 64 KB; entry ring 4 x 9 KB; bf16 tile ring 3 x 32 KB;
-// P 2 x 4 KB (64-byte swizzle); decode tables 1.5 KB.
+// Shared memory (219 KB): Q 64 KB; bf16 tile ring 2 x 64 KB; entry ring
+// 2 x 9 KB (32-token halves); P 8 KB (128-byte swizzle).
 //
-// Warp roles (320 threads): warp 0 loader (Q, entries), warp 1 MMA issuer and
-// TMEM owner, warps 2-5 dequant, warps 6-9 softmax + epilogue. Every wait is
+// Warp roles (448 threads): warp 0 loader (Q, entries), warp 1 MMA issuer and
+// TMEM owner, warps 2-9 dequant, warps 10-13 softmax + epilogue. Every wait is
 // bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -41,27 +46,27 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kLoaderWarp = 0, kMmaWarp = 1, kDeqWarp0 = 2, kSoftWarp0 = 6;
-constexpr int kTT = 32;                     // tokens per tile
+constexpr int kThreads = 448;
+constexpr int kDeqWarps = 8;
+constexpr int kLoaderWarp = 0, kMmaWarp = 1, kDeqWarp0 = 2, kSoftWarp0 = kDeqWarp0 + kDeqWarps;
+constexpr int kTT = 64;                     // tokens per tile
+constexpr int kHalf = 32;                   // tokens per entry copy
 constexpr int kRows = 64;                   // query rows per CTA
 constexpr int kEntry = 288;                 // bytes per FP4 entry (512 codes + 32 scales)
-constexpr int kRawStages = 4;
-constexpr int kRawStage = kTT * kEntry;     // 9216 B
-constexpr int kKStages = 3;
-constexpr int kKChunk = kTT * 128;          // 32 rows x 64 dims bf16 (4 KB)
-constexpr int kKStage = 8 * kKChunk;        // 32 KB
-constexpr int kPBufs = 2;
-constexpr int kPBuf = kRows * kTT * 2;      // 4 KB, 64-byte rows
-constexpr int kSBufs = 4;
+constexpr int kRawStages = 2;
+constexpr int kRawStage = kHalf * kEntry;   // 9216 B
+constexpr int kKStages = 2;
+constexpr int kKChunk = kTT * 128;          // 64 rows x 64 dims bf16 (8 KB)
+constexpr int kKStage = 8 * kKChunk;        // 64 KB
+constexpr int kPBuf = kRows * kTT * 2;      // 8 KB, 128-byte rows
+constexpr int kSBufs = 2;
+constexpr int kPrefetchHalves = 4;          // L2 prefetch distance (two tiles)
 
 constexpr int kOffQ = 0;
-constexpr int kOffRaw = kOffQ + 8 * 8192;
-constexpr int kOffK = kOffRaw + kRawStages * kRawStage;
-constexpr int kOffP = kOffK + kKStages * kKStage;
-constexpr int kOffLut2 = kOffP + kPBufs * kPBuf;     // 256 x u32: bf16x2 of a code byte's two nibbles
-constexpr int kOffLut1 = kOffLut2 + 1024;            // 256 x u16: bf16 of an E4M3 byte
-constexpr int kOffBar = kOffLut1 + 512;
+constexpr int kOffK = kOffQ + 8 * 8192;
+constexpr int kOffRaw = kOffK + kKStages * kKStage;
+constexpr int kOffP = kOffRaw + kRawStages * kRawStage;
+constexpr int kOffBar = kOffP + kPBuf;
 enum : int {
   B_QFULL = 0,
   B_RAWFULL = B_QFULL + 1,
@@ -71,8 +76,8 @@ enum : int {
   B_SFULL = B_KEMPTY + kKStages,
   B_SFREE = B_SFULL + kSBufs,
   B_PFULL = B_SFREE + kSBufs,
-  B_PVDONE = B_PFULL + kPBufs,
-  B_COUNT = B_PVDONE + kPBufs
+  B_PVDONE = B_PFULL + 1,
+  B_COUNT = B_PVDONE + 1
 };
 constexpr int kOffTmemPtr = kOffBar + B_COUNT * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
@@ -80,14 +85,14 @@ constexpr int kSmemBytes = kOffBar + 512;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 static_assert(kOffAbort + 4 <= kSmemBytes, "barrier area overflow");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kOffRaw % 1024 == 0 && kOffK % 1024 == 0 && kOffP % 1024 == 0, "1 KB swizzle atoms");
+static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0 && kOffRaw % 16 == 0, "operand alignment");
+static_assert(kTile % kTT == 0, "split ranges start on tile boundaries");
 
 constexpr uint32_t kColO = 0;               // O: columns 0-255, lanes 0-15 (dims 0-255) and 16-31 (256-511)
-constexpr uint32_t kColS = 256;             // S buffer i at columns 256 + 32 i, lanes 0-15
+constexpr uint32_t kColS = 256;             // S buffer i at columns 256 + 64 i, lanes 0-15
 constexpr uint32_t kTmemCols = 512;
 
 constexpr float kRescaleThreshold = 8.0f;
-static_assert(kTT == 32, "visibility is one 32-bit mask per tile");
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -114,6 +119,43 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// Byte permute with the sign-replicating selector mode (selector bit 3).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Eight E2M1 codes (byte k of x holds channel 2k in its low nibble and 2k+1
+// in its high nibble) to four bf16x2 words, exactly. The bf16 patterns of
+// the eight magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are split into a low-byte
+// and a high-byte table of 8 bytes each, indexed by the magnitude bits with
+// prmt; the sign byte is 0x80 or 0 from prmt's sign replication of the byte
+// whose top bit is the nibble's sign bit (x << 4 for even nibbles, x for odd).
+__device__ __forceinline__ void e2m1x8_to_bf16x2(uint32_t x, uint32_t (&w)[4]) {
+  constexpr uint32_t kLo03 = 0xC0800000u, kLo47 = 0xC0804000u;   // 00 00 80 C0 | 00 40 80 C0
+  constexpr uint32_t kHi03 = 0x3F3F3F00u, kHi47 = 0x40404040u;   // 00 3F 3F 3F | 40 40 40 40
+  const uint32_t x4 = x << 4;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t sel = (h ? (x >> 16) : x) & 0x7777u;
+    const uint32_t lo = prmt(kLo03, kLo47, sel);
+    const uint32_t sg = prmt(x4, x, h ? 0xFBEAu : 0xD9C8u);
+    const uint32_t hi = prmt(kHi03, kHi47, sel) | (sg & 0x80808080u);
+    w[2 * h] = prmt(lo, hi, 0x5140u);       // channels 4h, 4h+1
+    w[2 * h + 1] = prmt(lo, hi, 0x7362u);   // channels 4h+2, 4h+3
+  }
+}
+
+// One E4M3 scale byte as bf16x2 (both halves), exactly, through the
+// hardware FP8 -> f16 conversion (every E4M3 value is an f16 value).
+__device__ __forceinline__ __nv_bfloat162 e4m3_to_bf16x2(uint32_t byte) {
+  const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3);
+  const float f = __half2float(__half(hr));
+  const uint32_t w = pack_bf16(f, f);
+  return *reinterpret_cast<const __nv_bfloat162*>(&w);
+}
+
 // Page table entry of token t is usable (paged caches only).
 __device__ __forceinline__ bool page_ok(const DecodeParams& p, int b, int t) {
   if (!p.block_table) return true;
@@ -123,6 +165,30 @@ __device__ __forceinline__ bool page_ok(const DecodeParams& p, int b, int t) {
 
 __device__ __forceinline__ uint32_t swz128(int r, int u) {
   return (uint32_t)r * 128u + ((uint32_t)((u & 7) ^ (r & 7)) << 4);
+}
+
+// Source of the entry copy for tokens [t0, t0 + 32): the row pointer and the
+// number of entries (0 past a contiguous cache's end). A paged copy never
+// crosses a page (t0 is a multiple of 32, pages hold 64 tokens); a bad page
+// reads page 0, and the softmax masks its tokens.
+__device__ __forceinline__ const uint8_t* entry_src(const Fp4Params& P, const uint8_t* kvb, int b, int len,
+                                                    int t0, int& n, bool& bad) {
+  const DecodeParams& p = P.p;
+  bad = false;
+  if (P.paged) {
+    int pg = 0;
+    if (t0 < len) {
+      pg = p.block_table[(int64_t)b * p.max_pages + (t0 >> 6)];
+      if (pg < 0 || pg >= p.num_pages) {
+        bad = true;
+        pg = 0;
+      }
+    }
+    n = kHalf;
+    return kvb + ((int64_t)pg * 64 + (t0 & 63)) * kEntry;
+  }
+  n = min(kHalf, p.Lk - t0);
+  return kvb + (int64_t)b * p.kv_batch + (int64_t)(n > 0 ? t0 : 0) * kEntry;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __grid_constant__ Fp4Params P) {
@@ -138,33 +204,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   pdl_launch_dependents();
 
-  // decode tables (exact: E2M1 and E4M3 values are bf16 values)
-  {
-    uint32_t* lut2 = reinterpret_cast<uint32_t*>(smem + kOffLut2);
-    uint16_t* lut1 = reinterpret_cast<uint16_t*>(smem + kOffLut1);
-    for (int i = threadIdx.x; i < 256; i += kThreads) {
-      lut2[i] = pack_bf16(e2m1_value((uint32_t)i & 15u), e2m1_value((uint32_t)i >> 4));
-      lut1[i] = __bfloat16_as_ushort(__float2bfloat16_rn(e4m3_value((uint32_t)i)));
-    }
-  }
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
     for (int s = 0; s < kRawStages; ++s) {
       mbar_init(bar(B_RAWFULL + s), 1);
-      mbar_init(bar(B_RAWEMPTY + s), 4);   // one arrival per dequant warp
+      mbar_init(bar(B_RAWEMPTY + s), kDeqWarps);   // one arrival per dequant warp
     }
     for (int s = 0; s < kKStages; ++s) {
-      mbar_init(bar(B_KFULL + s), 4);      // one arrival per dequant warp
+      mbar_init(bar(B_KFULL + s), kDeqWarps);      // one arrival per dequant warp
       mbar_init(bar(B_KEMPTY + s), 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
       mbar_init(bar(B_SFREE + i), 1);
     }
-    for (int i = 0; i < kPBufs; ++i) {
-      mbar_init(bar(B_PFULL + i), 1);
-      mbar_init(bar(B_PVDONE + i), 1);
-    }
+    mbar_init(bar(B_PFULL), 1);
+    mbar_init(bar(B_PVDONE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -196,84 +251,96 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
       const int qrow = b * p.HQ + rb * kRows;
       mbar_arrive_expect_tx(bar(B_QFULL), 8 * 8192);
       for (int c = 0; c < 8; ++c) tma_load_2d(sb0 + kOffQ + c * 8192, &P.tm_q, bar(B_QFULL), 64 * c, qrow);
+      const int nh = 2 * ntiles;
+      for (int hj = 0; hj < kPrefetchHalves && hj < nh; ++hj) {
+        int n;
+        bool bad;
+        const uint8_t* src = entry_src(P, kvb, b, len, t_begin + kHalf * hj, n, bad);
+        if (n > 0) prefetch_l2_bulk(src, (uint32_t)(n * kEntry));
+      }
       bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int s = j % kRawStages;
-        if (j >= kRawStages && !mbar_wait(bar(B_RAWEMPTY + s), ((j / kRawStages) - 1) & 1)) {
+      for (int hj = 0; hj < nh && ok; ++hj) {
+        const int s = hj % kRawStages;
+        if (hj >= kRawStages && !mbar_wait(bar(B_RAWEMPTY + s), ((hj / kRawStages) - 1) & 1)) {
           ok = false;
           break;
         }
-        const int t0 = t_begin + j * kTT;
-        const uint8_t* src;
-        int n = kTT;
-        if (P.paged) {
-          int pg = 0;
-          if (t0 < len) {
-            pg = p.block_table[(int64_t)b * p.max_pages + (t0 >> 6)];
-            if (pg < 0 || pg >= p.num_pages) {
-              flag_error(p, MLA_DEVICE_ERR_BLOCK_TABLE);
-              pg = 0;   // its tokens are masked by the softmax
-            }
-          }
-          src = kvb + ((int64_t)pg * 64 + (t0 & 63)) * kEntry;
+        int n;
+        bool bad;
+        const uint8_t* src = entry_src(P, kvb, b, len, t_begin + kHalf * hj, n, bad);
+        if (bad) flag_error(p, MLA_DEVICE_ERR_BLOCK_TABLE);
+        if (n > 0) {
+          mbar_arrive_expect_tx(bar(B_RAWFULL + s), (uint32_t)(n * kEntry));
+          bulk_load(sb0 + kOffRaw + s * kRawStage, src, (uint32_t)(n * kEntry), bar(B_RAWFULL + s));
         } else {
-          src = kvb + (int64_t)b * p.kv_batch + (int64_t)t0 * kEntry;
-          n = min(kTT, p.Lk - t0);   // stay inside this sequence's rows
+          mbar_arrive(bar(B_RAWFULL + s));   // nothing left in the cache: rows are zero-filled
         }
-        mbar_arrive_expect_tx(bar(B_RAWFULL + s), (uint32_t)(n * kEntry));
-        bulk_load(sb0 + kOffRaw + s * kRawStage, src, (uint32_t)(n * kEntry), bar(B_RAWFULL + s));
+        const int hp = hj + kPrefetchHalves;
+        if (hp < nh) {
+          const uint8_t* ps = entry_src(P, kvb, b, len, t_begin + kHalf * hp, n, bad);
+          if (n > 0) prefetch_l2_bulk(ps, (uint32_t)(n * kEntry));
+        }
         if (*abort_flag) ok = false;
       }
       if (!ok) fail();
     }
     __syncwarp();
-  } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + 4) {
+  } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + kDeqWarps) {
     // ------------------------------------------------------------------ dequant
-    // 2048 pieces of 8 channels per tile, 16 per thread: piece i = token
-    // i/64, chunk (i/8)%8, 16-byte unit i%8 (channels 64 chunk + 8 unit)
-    const int dt = threadIdx.x - kDeqWarp0 * 32;   // 0..127
-    const uint32_t* lut2 = reinterpret_cast<const uint32_t*>(smem + kOffLut2);
-    const uint16_t* lut1 = reinterpret_cast<const uint16_t*>(smem + kOffLut1);
+    // Per 32-token half: 2048 pieces of 8 channels, 8 per thread: piece i =
+    // token i/64, chunk (i/8)%8, 16-byte unit i%8 (channels 64 chunk + 8 unit).
+    // A warp covers one token's 4 chunks x 8 units: whole 128-byte rows, so
+    // both the entry reads and the swizzled tile stores are conflict-free.
+    const int dt = threadIdx.x - kDeqWarp0 * 32;   // 0..255
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int rs = j % kRawStages, ks = j % kKStages;
-      bool got = mbar_wait(bar(B_RAWFULL + rs), (j / kRawStages) & 1);
-      if (got && j >= kKStages) got = mbar_wait(bar(B_KEMPTY + ks), ((j / kKStages) - 1) & 1);
+      const int ks = j % kKStages;
+      bool got = j < kKStages || mbar_wait(bar(B_KEMPTY + ks), ((j / kKStages) - 1) & 1);
+      got = __all_sync(0xffffffffu, got) != 0;
+      const uint32_t kbase = kOffK + ks * kKStage;
+      for (int h = 0; h < 2 && got; ++h) {
+        const int hj = 2 * j + h, rs = hj % kRawStages;
+        got = mbar_wait(bar(B_RAWFULL + rs), (hj / kRawStages) & 1);
+        if (!__all_sync(0xffffffffu, got)) {
+          got = false;
+          break;
+        }
+        const uint8_t* rawp = smem + kOffRaw + rs * kRawStage;
+        const int t0 = t_begin + kHalf * hj;
+        constexpr int kPieces = 2048 / (32 * kDeqWarps);
+        uint32_t cw[kPieces], sb[kPieces];
+#pragma unroll
+        for (int k = 0; k < kPieces; ++k) {
+          const int i = dt + 32 * kDeqWarps * k, t = i >> 6, c = (i >> 3) & 7, u = i & 7;
+          const uint8_t* e = rawp + t * kEntry;
+          cw[k] = *reinterpret_cast<const uint32_t*>(e + 32 * c + 4 * u);
+          sb[k] = e[256 + 4 * c + (u >> 1)];
+        }
+#pragma unroll
+        for (int k = 0; k < kPieces; ++k) {
+          const int i = dt + 32 * kDeqWarps * k, t = i >> 6, c = (i >> 3) & 7, u = i & 7;
+          // rows past the sequence (stale or never loaded) become zeros
+          const __nv_bfloat162 s2 = (t0 + t < len) ? e4m3_to_bf16x2(sb[k]) : __float2bfloat162_rn(0.f);
+          uint32_t w[4];
+          e2m1x8_to_bf16x2(cw[k], w);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]), s2);
+            w[q] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          *reinterpret_cast<uint4*>(smem + kbase + c * kKChunk + swz128(kHalf * h + t, u)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_RAWEMPTY + rs));
+      }
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
-      const uint8_t* rawp = smem + kOffRaw + rs * kRawStage;
-      const uint32_t kbase = sb0 + kOffK + ks * kKStage;
-      const int t0 = t_begin + j * kTT;
-#pragma unroll 4
-      for (int k = 0; k < 16; ++k) {
-        const int i = dt + 128 * k, t = i >> 6, c = (i >> 3) & 7, u = i & 7;
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (t0 + t < len) {
-          const uint8_t* e = rawp + t * kEntry;
-          const uint32_t codes = *reinterpret_cast<const uint32_t*>(e + 32 * c + 4 * u);
-          const uint32_t sc = lut1[e[256 + 4 * c + (u >> 1)]];
-          const __nv_bfloat162 s2 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)sc),
-                                                       __ushort_as_bfloat16((unsigned short)sc));
-          uint32_t w[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t pr = lut2[(codes >> (8 * q)) & 0xffu];
-            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pr);
-            const __nv_bfloat162 m = __hmul2(v, s2);
-            w[q] = *reinterpret_cast<const uint32_t*>(&m);
-          }
-          out = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        *reinterpret_cast<uint4*>(smem + (kbase - sb0) + c * kKChunk + swz128(t, u)) = out;
-      }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(B_KFULL + ks));
-        mbar_arrive(bar(B_RAWEMPTY + rs));
-      }
+      if (lane == 0) mbar_arrive(bar(B_KFULL + ks));
       if (*abort_flag) ok = false;
       ok = __all_sync(0xffffffffu, ok) != 0;
     }
@@ -284,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
       const uint32_t idesc_qk = idesc_bf16_f32(kRows, kTT, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);
       const uint64_t qd = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
+      const uint64_t pd = smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
       bool ok = mbar_wait(bar(B_QFULL), 0);
       int qj = 0, pj = 0;
       uint64_t t_idle = global_ns();
@@ -296,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
           if (sfree && mbar_poll(bar(B_KFULL + ks), (qj / kKStages) & 1)) {
             tc_fence_after();
             const uint64_t kd = smem_desc(sb0 + kOffK + ks * kKStage, 16, 1024, kSwizzle128B);
-            const uint32_t d = tmem + kColS + 32u * sbuf;
+            const uint32_t d = tmem + kColS + 64u * sbuf;
 #pragma unroll
             for (int kk = 0; kk < 32; ++kk) {
               const int c = kk >> 2, sub = kk & 3;
@@ -308,39 +376,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
             prog = true;
           }
         }
-        if (pj < qj) {
-          const int pb = pj % kPBufs, ks = pj % kKStages;
-          if (mbar_poll(bar(B_PFULL + pb), (pj / kPBufs) & 1)) {
-            tc_fence_after();
-            const uint64_t vd = smem_desc(sb0 + kOffK + ks * kKStage, kKChunk, 1024, kSwizzle128B);
-            const uint64_t pd = smem_desc(sb0 + kOffP + pb * kPBuf, 16, 512, kSwizzle64B);
+        if (pj < qj && mbar_poll(bar(B_PFULL), pj & 1)) {
+          tc_fence_after();
+          const int ks = pj % kKStages;
+          const uint64_t vd = smem_desc(sb0 + kOffK + ks * kKStage, kKChunk, 1024, kSwizzle128B);
 #pragma unroll
-            for (int n = 0; n < 2; ++n) {
+          for (int n = 0; n < 2; ++n) {
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {
-                // P: 16 tokens per step (K-major, 64-byte rows); V: the tile's
-                // chunks 4n..4n+3 (MN-major); D: lanes 16n.. of each subpartition
-                mma_bf16_ss(tmem + ((16u * n) << 16) + kColO, desc_advance(pd, 32 * kk),
-                            desc_advance(vd, 4 * n * kKChunk + 2048 * kk), idesc_pv,
-                            (pj > 0 || kk > 0) ? 1u : 0u);
-              }
+            for (int kk = 0; kk < 4; ++kk) {
+              // P: 16 tokens per step (K-major, 128-byte rows); V: the tile's
+              // chunks 4n..4n+3 (MN-major); D: lanes 16n.. of each subpartition
+              mma_bf16_ss(tmem + ((16u * n) << 16) + kColO, desc_advance(pd, 32 * kk),
+                          desc_advance(vd, 4 * n * kKChunk + 2048 * kk), idesc_pv,
+                          (pj > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(bar(B_KEMPTY + ks));
-            mma_commit(bar(B_PVDONE + pb));
-            ++pj;
-            prog = true;
           }
+          mma_commit(bar(B_KEMPTY + ks));
+          mma_commit(bar(B_PVDONE));
+          ++pj;
+          prog = true;
         }
         if (prog) {
           idle = 0;
-        } else {
-          // nothing ready: yield the issue slots this sub-partition shares
-          // with a dequant and a softmax warp
-          __nanosleep(64);
-          if ((++idle & 255u) == 0) {
-            if (idle == 256u) t_idle = global_ns();
-            else if (global_ns() - t_idle > 1000000000ull || *abort_flag) ok = false;
-          }
+        } else if ((++idle & 255u) == 0) {
+          if (idle == 256u) t_idle = global_ns();
+          else if (global_ns() - t_idle > 1000000000ull || *abort_flag) ok = false;
         }
       }
       if (!ok) fail();
@@ -366,24 +426,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
     float m_run = -INFINITY, l_run = 0.f;
     bool ab = false;
     auto wait_pv = [&](int t) {
-      if (!ab) ab = !mbar_wait(bar(B_PVDONE + (t % kPBufs)), (t / kPBufs) & 1);
+      if (!ab) ab = !mbar_wait(bar(B_PVDONE), t & 1);
     };
     for (int j = 0; j < ntiles; ++j) {
-      const int sbuf = j % kSBufs, pb = j % kPBufs;
+      const int sbuf = j % kSBufs;
       if (!ab) ab = !mbar_wait(bar(B_SFULL + sbuf), (j / kSBufs) & 1);
       ab = __any_sync(0xffffffffu, ab);
       float s[kTT];
       if (!ab) {
         tc_fence_after();
-        uint32_t v[2][16];
-        tmem_ld16(tmem + lane_base + kColS + 32u * sbuf, v[0]);
-        tmem_ld16(tmem + lane_base + kColS + 32u * sbuf + 16u, v[1]);
+        uint32_t v[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_base + kColS + 64u * sbuf + 16u * c, v[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          s[i] = __uint_as_float(v[0][i]);
-          s[16 + i] = __uint_as_float(v[1][i]);
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(v[c][i]);
       } else {
 #pragma unroll
         for (int i = 0; i < kTT; ++i) s[i] = 0.f;
@@ -395,18 +454,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
       const int tb = t_begin + j * kTT;
       int lim = t_end - tb;
       if (causal) lim = min(lim, causal_last - tb + 1);
-      if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;
+      if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;   // a tile is one page
       if (ab) lim = 0;
-      // visibility of the tile's 32 tokens as a bit mask: the question's mask
+      // visibility of the tile's 64 tokens as bit masks: the question's mask
       // is read once per token, one lane each (tb is the same for every row)
-      uint32_t vbits = lim >= kTT ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
-      if (mask != nullptr) vbits &= __ballot_sync(0xffffffffu, tb + lane < t_end && mask[tb + lane] != 0);
-      float mx = -INFINITY;
+      uint32_t v0 = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+      uint32_t v1 = lim >= 64 ? 0xffffffffu : (lim <= 32 ? 0u : (1u << (lim - 32)) - 1u);
+      if (mask != nullptr) {
+        v0 &= __ballot_sync(0xffffffffu, tb + lane < t_end && mask[tb + lane] != 0);
+        v1 &= __ballot_sync(0xffffffffu, tb + 32 + lane < t_end && mask[tb + 32 + lane] != 0);
+      }
+      // eight independent partial maxima and sums keep the dependency chains short
+      float mp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mp[i] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kTT; ++c) {
-        s[c] = ((vbits >> c) & 1u) ? s[c] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        const uint32_t vb = c < 32 ? v0 : v1;
+        s[c] = ((vb >> (c & 31)) & 1u) ? s[c] * sl2 : -INFINITY;
+        mp[c & 7] = fmaxf(mp[c & 7], s[c]);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_new = fmaxf(m_run, mx);
       const bool need = (m_new - m_run) > kRescaleThreshold;
       float alpha = 1.f;
@@ -415,30 +484,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
         m_run = m_new;
       }
       uint32_t pk[kTT / 2];
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       const bool none = (m_run == -INFINITY);
 #pragma unroll
       for (int c = 0; c < kTT / 2; ++c) {
         const float p0 = none ? 0.f : fast_exp2(s[2 * c] - m_run);
         const float p1 = none ? 0.f : fast_exp2(s[2 * c + 1] - m_run);
-        psum += p0 + p1;
+        ps[c & 3] += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
-      l_run = l_run * alpha + psum;
+      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       // lanes 16-31 rescale the second half of the same rows: take lane i's alpha
       const float alpha_row = __shfl_sync(0xffffffffu, alpha, lane & 15);
       const bool need_row = __shfl_sync(0xffffffffu, need, lane & 15);
 
-      if (j >= kPBufs) wait_pv(j - kPBufs);
+      // P and O are free once PV(j - 1) has completed
+      if (j >= 1) wait_pv(j - 1);
       if (hi == 0) {
-        uint8_t* prow = smem + kOffP + pb * kPBuf + m * 64;
+        uint8_t* prow = smem + kOffP + m * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + 16 * (c ^ ((m >> 1) & 3))) =
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + 16 * (c ^ (m & 7))) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       if (__any_sync(0xffffffffu, need_row && j > 0)) {
-        wait_pv(j - 1);
         ab = __any_sync(0xffffffffu, ab);
         if (!ab) {
           tc_fence_after();
@@ -463,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(1, 128);   // P(j) of every row is written
-      if (leader) mbar_arrive(bar(B_PFULL + pb));
+      if (leader) mbar_arrive(bar(B_PFULL));
     }
 
     // ---------------------------------------------------------------- epilogue
