@@ -240,24 +240,32 @@ class ClockSampler:
                 "samples": len(sm), "source": "nvml" if self.samples else "nvidia-smi"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the named csrc files (the profiled kernel's own sources)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "latent_kv_decode_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in sorted(files):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes per decode launch from the committed ncu summary, if the
+    summary's kernel sources still hash to the value it was captured with."""
     p = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
+    m_files = re.search(r"kernel sources:\s*(.+)", txt)
     m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
     m_bytes = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", txt)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_files or not m_hash or not m_bytes:
+        return None
+    files = m_files.group(1).replace("`", "").split()
+    try:
+        if m_hash.group(1) != kernel_source_hash(files):
+            return None
+    except OSError:
         return None
     return float(m_bytes.group(1))
 
