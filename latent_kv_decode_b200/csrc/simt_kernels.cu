@@ -351,6 +351,114 @@ __global__ void __launch_bounds__(128) combine_simt(DecodeParams p) {
   if (p.lse && threadIdx.x == 0) p.lse[grow] = red[0];
 }
 
+// combine, warp per row: for Ckv = 32 * kCols. The splits' lse values are
+// reduced across lanes; lane i owns columns [kCols i, kCols i + kCols) and
+// issues all its 16-byte partial-O loads of a group of splits before using
+// them, so a row costs a few memory latencies rather than one per split.
+template <typename TQ, int kCols>
+__global__ void __launch_bounds__(128) combine_warp(DecodeParams p) {
+  constexpr int kSplitGroup = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t grow = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);   // b * HQ + r
+  if (grow >= (int64_t)p.B * p.HQ) return;                             // whole warp
+  const int b = (int)(grow / p.HQ), r = (int)(grow % p.HQ);
+  const int h = r / p.Q, q = r % p.Q;
+  const int S = p.num_splits;
+  const int64_t sstride = (int64_t)p.B * p.HQ;
+  float m = p.sinks ? p.sinks[h] : -INFINITY;
+  for (int s = lane; s < S; s += 32) m = fmaxf(m, p.ws_lse[s * sstride + grow]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float den = 0.f;
+  if (m != -INFINITY) {
+    for (int s = lane; s < S; s += 32) {
+      const float l = p.ws_lse[s * sstride + grow];
+      den += (l == -INFINITY) ? 0.f : expf(l - m);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (p.sinks) den += expf(p.sinks[h] - m);
+  }
+  const float L = den > 0.f ? m + logf(den) : -INFINITY;
+
+  const int c0 = lane * kCols;
+  float acc[kCols];
+#pragma unroll
+  for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += kSplitGroup) {
+    float4 v[kSplitGroup][kCols / 4];
+    float w[kSplitGroup];
+#pragma unroll
+    for (int g = 0; g < kSplitGroup; ++g) {
+      const int s = min(s0 + g, S - 1);
+      const float l = p.ws_lse[s * sstride + grow];
+      w[g] = (s0 + g >= S || l == -INFINITY || L == -INFINITY) ? 0.f : expf(l - L);
+      const float4* src = reinterpret_cast<const float4*>(p.ws_o + (s * sstride + grow) * p.Ckv + c0);
+#pragma unroll
+      for (int i = 0; i < kCols / 4; ++i) v[g][i] = src[i];
+    }
+#pragma unroll
+    for (int g = 0; g < kSplitGroup; ++g) {
+      if (w[g] == 0.f) continue;
+#pragma unroll
+      for (int i = 0; i < kCols / 4; ++i) {
+        acc[4 * i] = fmaf(w[g], v[g][i].x, acc[4 * i]);
+        acc[4 * i + 1] = fmaf(w[g], v[g][i].y, acc[4 * i + 1]);
+        acc[4 * i + 2] = fmaf(w[g], v[g][i].z, acc[4 * i + 2]);
+        acc[4 * i + 3] = fmaf(w[g], v[g][i].w, acc[4 * i + 3]);
+      }
+    }
+  }
+  if (p.rope_tail > 0) {
+    const int pos = seq_len_of(p, b) - p.Q + q;
+    const int base = p.Ckv - p.rope_tail;
+    if (p.rope_tail <= 64) {
+      // lane j evaluates pair j's rotation once (the same double-precision
+      // angle as inverse_rope_pair); the lanes owning the tail take it by shuffle
+      double cj = 1.0, sj = 0.0;
+      if (2 * lane < p.rope_tail) {
+        const double freq = pow((double)p.rope_theta, -2.0 * (double)lane / (double)p.rope_tail);
+        sincos(-(double)pos * freq, &sj, &cj);
+      }
+#pragma unroll
+      for (int i = 0; i < kCols; i += 2) {
+        const int c = c0 + i;
+        const int jp = c >= base ? (c - base) >> 1 : 0;
+        const double cr = __shfl_sync(0xffffffffu, cj, jp), sr = __shfl_sync(0xffffffffu, sj, jp);
+        if (c >= base) {
+          const float fa = acc[i], fb = acc[i + 1];
+          acc[i] = (float)(fa * cr - fb * sr);
+          acc[i + 1] = (float)(fa * sr + fb * cr);
+        }
+      }
+    } else if (c0 + kCols > base) {
+#pragma unroll
+      for (int i = 0; i < kCols; i += 2) {
+        const int c = c0 + i;
+        if (c >= base) inverse_rope_pair(acc[i], acc[i + 1], (c - base) >> 1, p.rope_tail, p.rope_theta, pos);
+      }
+    }
+  }
+  TQ* xo = reinterpret_cast<TQ*>(p.x) + grow * p.Ckv + c0;
+  if constexpr (sizeof(TQ) == 2) {
+#pragma unroll
+    for (int i = 0; i < kCols; i += 8) {
+      uint32_t u[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 t = __floats2bfloat162_rn(acc[i + 2 * k], acc[i + 2 * k + 1]);
+        u[k] = *reinterpret_cast<const uint32_t*>(&t);
+      }
+      *reinterpret_cast<uint4*>(xo + i) = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kCols; i += 4)
+      *reinterpret_cast<float4*>(xo + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+  }
+  if (p.lse && lane == 0) p.lse[grow] = L;
+}
+
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
@@ -406,8 +514,25 @@ cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaS
   return bf16 ? decode_launch<__nv_bfloat16, false>(p, st) : decode_launch<float, false>(p, st);
 }
 
+template <typename TQ>
+static cudaError_t combine_warp_launch(const DecodeParams& p, cudaStream_t st) {
+  const unsigned grid = (unsigned)(((int64_t)p.B * p.HQ + 3) / 4);
+  switch (p.Ckv) {
+    case 128: combine_warp<TQ, 4><<<grid, 128, 0, st>>>(p); break;
+    case 256: combine_warp<TQ, 8><<<grid, 128, 0, st>>>(p); break;
+    default: combine_warp<TQ, 16><<<grid, 128, 0, st>>>(p); break;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t st) {
   const int64_t rows = (int64_t)p.B * p.HQ;
+  // 16-byte loads and stores: the partials and outputs are row-contiguous
+  // with rows of Ckv elements, and the buffers come from the allocator
+  const bool vec = (p.Ckv == 128 || p.Ckv == 256 || p.Ckv == 512) &&
+                   (reinterpret_cast<uintptr_t>(p.ws_o) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.x) & 15u) == 0 && (p.rope_tail & 1) == 0;
+  if (vec) return bf16 ? combine_warp_launch<__nv_bfloat16>(p, st) : combine_warp_launch<float>(p, st);
   if (bf16)
     combine_simt<__nv_bfloat16><<<(unsigned)rows, 128, 0, st>>>(p);
   else
