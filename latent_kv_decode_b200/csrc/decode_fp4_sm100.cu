@@ -560,6 +560,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
       scale_o = lfin > 0.f ? w / lfin : 0.f;
       lse = lfin > 0.f ? (mfin + log2f(lfin)) * kLn2 : -INFINITY;
     }
+    // Inverse RoPE of an unsplit row block: with Q = 1 every row of the CTA
+    // sits at position len - 1, so lane j evaluates tail pair j's rotation
+    // once (the double-precision angle of inverse_rope_pair) and the lanes
+    // holding the tail take it by shuffle, instead of each tail lane
+    // evaluating all of its pairs in turn.
+    const int rope_base = p.Ckv - p.rope_tail;
+    const bool rope_shared = p.num_splits == 1 && p.rope_tail > 0 && p.rope_tail <= 64 && p.Q == 1;
+    double rope_c = 1.0, rope_s = 0.0;
+    if (rope_shared && 2 * lane < p.rope_tail) {
+      const double freq = pow((double)p.rope_theta, -2.0 * (double)lane / (double)p.rope_tail);
+      sincos(-(double)(len - 1) * freq, &rope_s, &rope_c);
+    }
 #pragma unroll 1
     for (int c = 0; c < 16; ++c) {
       uint32_t v[16];
@@ -580,7 +592,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp4_sm100_kernel(const __g
         for (int i = 0; i < 16; i += 4)
           *reinterpret_cast<float4*>(o + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
       } else {
-        if (p.rope_tail > 0 && col >= p.Ckv - p.rope_tail) {
+        if (rope_shared) {
+          if (256 + 16 * c + 16 > rope_base) {   // the same test in every lane: all shuffle
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              const int cc = col + i;
+              const int jp = cc >= rope_base ? (cc - rope_base) >> 1 : 0;
+              const double cr = __shfl_sync(0xffffffffu, rope_c, jp);
+              const double sr = __shfl_sync(0xffffffffu, rope_s, jp);
+              if (cc >= rope_base) {
+                const float fa = f[i], fb = f[i + 1];
+                f[i] = (float)(fa * cr - fb * sr);
+                f[i + 1] = (float)(fa * sr + fb * cr);
+              }
+            }
+          }
+        } else if (p.rope_tail > 0 && col >= rope_base) {
           const int pos = len - p.Q + q;
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
