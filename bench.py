@@ -240,12 +240,39 @@ class ClockSampler:
                 "samples": len(sm), "source": "nvml" if self.samples else "nvidia-smi"}
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed, so
+    that documentation edits do not count as a change of the profiled code.
+    String and character literals are kept as they are."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(files) -> str:
-    """Hash of the named csrc files (the profiled kernel's own sources)."""
+    """Hash of the code (comments stripped) of the named csrc files: the
+    profiled kernel's own sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "latent_kv_decode_b200", "csrc")
     for f in sorted(files):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(_code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -4,8 +4,8 @@
 //
 // One 2-CTA cluster per (128-row block, sequence, split). CTA r of the pair
 // owns query rows [64r, 64r+64) of the block; every MMA is a pair MMA
-// (tcgen05 cta_group::2, M = 128), so each SM computes its own 64 rows at the
-// full datapath width. Per 128-token tile of the cache:
+// (tcgen05 cta_group::2, M = 128), so each SM computes its own 64 rows and the
+// pair shares one K tile. Per 128-token tile of the cache:
 //
 //   S  = Q . K^T   over the 576 dims in 64-dim chunks (8 latent + 1 rope).
 //                  CTA r supplies tokens [64r, 64r+64) of the tile (the N half
@@ -17,9 +17,10 @@
 //                  for all 128 tokens.
 //
 // The latent rows are therefore read twice per tile (once as K, once as V,
-// cut differently between the pair); the K producer prefetches whole row
-// ranges into L2 three tiles ahead, so HBM sees each cache row once and both
-// shared-memory loads are L2 hits. Every TMA request moves 64 rows x 2 chunks
+// cut differently between the pair); the V read follows the K read of the
+// same rows closely enough to hit in L2, so HBM sees each cache row once (an
+// explicit L2 prefetch ahead of the K producer measured no gain and is off,
+// kPrefetchTiles = 0). Every TMA request moves 64 rows x 2 chunks
 // (16 KB) through a 4-D view of the cache whose box lands already in the
 // 128-byte-swizzled layout the MMAs read. Scores and the output accumulator
 // live in TMEM (S double-buffered: 2 x 64 columns; O: 2 x 128 columns).

@@ -6,7 +6,9 @@
 //   up_proj_simt    out   = W_UV[h] . x                       (blank [5])
 //   decode_simt     scores, scale, mask, online softmax, latent aggregation
 //                   (blanks [2]-[4], step 5), FP4 entries, sinks, inverse RoPE
-//   combine_simt    log-sum-exp merge of split partials + epilogue
+//   combine_warp    log-sum-exp merge of split partials + epilogue, a warp
+//                   per row (Ckv 128 / 256 / 512, 16-byte aligned buffers)
+//   combine_simt    the same merge for any other shape
 //
 // All arithmetic is float32; inputs are float32 or bf16 (converted on load).
 #include "common.cuh"

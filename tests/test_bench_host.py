@@ -29,3 +29,19 @@ def test_algorithmic_bytes_of_the_dsv3_step():
     assert a["step_bytes"] == 340_787_200
     # QK 576-wide + PV 512-wide per (row, token); absorb + up-projection per row
     assert a["step_flops"] == 2 * 64 * 128 * 4096 * (576 + 512) + 2 * 64 * 128 * 512 * (128 + 128)
+
+
+def test_code_hash_ignores_comments_but_not_code():
+    src = 'int a = 1; // note\n/* block */ const char* s = "x // kept";\n'
+    assert bench._code_only(src) == bench._code_only(src.replace("note", "other note"))
+    assert bench._code_only(src) != bench._code_only(src.replace("a = 1", "a = 2"))
+    assert '"x // kept"' in bench._code_only(src)
+
+
+def test_committed_profiles_match_the_current_kernel_code():
+    # each decode summary names its kernel's sources and the hash of their code
+    # when it was captured; the bench reports its traffic only while they match
+    for workload, lo, hi in [("dsv3_b64_lk4096", 3.0e8, 3.4e8), ("v41_fp4_sink_h64", 7.5e7, 9.0e7)]:
+        t = bench.profiled_traffic(workload)
+        assert t is not None, f"profiles/decode_{workload}.md is stale for the current kernel code"
+        assert lo <= t <= hi
