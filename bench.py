@@ -45,6 +45,15 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode tokens/s and achieved HBM TB/s (% of roofline) per MLA layer, 1×B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the datasheet figures, reported beside the measured-peak fractions
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def spec_fraction(achieved: float, unit: str) -> float:
+    """achieved / the datasheet peak of its unit (HBM GB/s or dense bf16 TFLOP/s)."""
+    return achieved / (SPEC_PEAKS["hbm_gbs"] if unit == "GB/s" else SPEC_PEAKS["bf16_tflops"])
+
+
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -489,6 +498,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         ),
         "step": {
             "bytes": int(alg["step_bytes"]), "flops": int(alg["step_flops"]),
+            "roofline_frac_of_spec": round(
+                max(alg["step_bytes"] / (SPEC_PEAKS["hbm_gbs"] * 1e9),
+                    alg["step_flops"] / (SPEC_PEAKS["bf16_tflops"] * 1e12)) / (mean_step * 1e-3), 4),
             "TB_per_s": round(step_gbs / 1e3, 4), "TFLOP_per_s": round(step_tf, 2),
             "roofline_us": round(roof_s * 1e6, 2),
             "roofline_frac": round(roof_s / (mean_step * 1e-3), 4),
@@ -513,6 +525,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clk.summary(),
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": tflops, "source": psrc},
     }
+    r = res["roofline"]
+    r["frac_of_spec"] = round(spec_fraction(r["achieved"], r["unit"]), 4)
     return res
 
 

@@ -57,3 +57,8 @@ def test_committed_profiles_match_the_current_kernel_code():
             assert lo <= t <= hi
     if stale:
         pytest.xfail(f"profile summaries older than the kernel code: {stale}")
+
+
+def test_spec_fraction_uses_the_datasheet_peak_of_the_unit():
+    assert abs(bench.spec_fraction(4000.0, "GB/s") - 0.5) < 1e-12
+    assert abs(bench.spec_fraction(1125.0, "TFLOP/s") - 0.5) < 1e-12
