@@ -36,7 +36,9 @@ CacheDecompressed form of the ackingliu.top "DeepSeek MLA projection
 absorption" article) on tiny inputs; rows of the softmax sum to 1; masked
 weights are exactly 0; single-visible-token and zero-query closed forms;
 Lk = 1 closed form; W_UK/W_UV row-split closed forms; Q=2 causal prefix
-property; split-merge invariance; paged == contiguous.
+property; split-merge invariance; paged == contiguous. Cache append
+(tests/test_oracle_append.py): token-by-token appends read back by
+gather_paged equal the rows in order; untouched slots keep their bytes.
 """
 from __future__ import annotations
 
@@ -224,6 +226,34 @@ def gather_paged(pool, block_table, seq_lens, page_size: int, Lk: int | None = N
     for b in range(B):
         for t in range(int(L[b])):
             out[b, t] = pool[bt[b, t // page_size], t % page_size]
+    return out
+
+
+def cache_append(pool, block_table, seq_lens, rows, page_size: int):
+    """Write each sequence's Q new cache rows into their paged slots.
+
+    rows (B, Q, C) are the new tokens' rows (latent, rope part, combined row
+    or FP4 entry); seq_lens are the lengths after the append, so new token i
+    of sequence b sits at position t = seq_lens[b] - Q + i and goes to row
+    t mod page_size of page block_table[b][t div page_size] -- the slot
+    addressing read back by gather_paged (the neuronix page appends the new
+    token's latent to the LatentKVCachePool before attending). Returns a new
+    pool of the input's dtype; a page id outside [0, num_pages) raises.
+    """
+    out = np.array(pool, copy=True)
+    bt = np.asarray(block_table)
+    L = np.asarray(seq_lens, np.int64)
+    r = np.asarray(rows)
+    B, Q = r.shape[0], r.shape[1]
+    for b in range(B):
+        for i in range(Q):
+            t = int(L[b]) - Q + i
+            if t < 0:
+                raise ValueError(f"sequence {b}: length {int(L[b])} shorter than the {Q} new tokens")
+            page = int(bt[b, t // page_size])
+            if not 0 <= page < out.shape[0]:
+                raise ValueError(f"sequence {b}, token {t}: page id {page} outside the pool")
+            out[page, t % page_size] = r[b, i]
     return out
 
 

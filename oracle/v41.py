@@ -39,7 +39,8 @@ set (tests/golden/e2m1_values.json); nearest-even ties of the quantiser;
 FP4 round-trip error bound on N(0,1) latents; 288 B per entry and cache
 bytes independent of H; RoPE against complex multiplication by
 e^{i pos theta_j}, relative-position property, identity at pos 0, round trip
-and untouched head dims; the sink's closed form with uniform logits.
+and untouched head dims; the sink's closed form with uniform logits;
+token-by-token FP4 appends equal cache_write of the whole sequence.
 """
 from __future__ import annotations
 
@@ -165,6 +166,22 @@ def cache_write(latent, tail: int = 64, theta: float = 10000.0):
     Lk = lat.shape[1]
     pos = np.broadcast_to(np.arange(Lk, dtype=F64)[None, :], lat.shape[:2])
     return fp4_quantize(rope_tail(lat, pos, tail, theta))
+
+
+def fp4_cache_append(pool, block_table, seq_lens, latent_new, page_size: int = 64, tail: int = 64,
+                     theta: float = 10000.0):
+    """Shared-latent cache append into a paged pool of 288-byte entries.
+
+    latent_new (B, Q, 512): the new tokens' latents; seq_lens: lengths after
+    the append. Each new token's tail is rotated at its position
+    seq_lens[b] - Q + i, quantised to an FP4 entry, and written to its slot
+    (mla.cache_append's addressing): the per-token form of cache_write.
+    """
+    lat = np.asarray(latent_new, F64)
+    B, Q, D = lat.shape
+    pos = np.asarray(seq_lens, np.int64)[:, None] - Q + np.arange(Q)[None, :]
+    ent = fp4_quantize(rope_tail(lat, pos.astype(F64), tail, theta), D)
+    return _mla.cache_append(pool, block_table, seq_lens, ent, page_size)
 
 
 def shared_latent_decode(q, entries, sinks, softmax_scale, seq_lens=None, causal: bool = False,

@@ -116,3 +116,40 @@ def test_wrong_rope_frequency_is_caught():
     z = (x[:, 448::2] + 1j * x[:, 449::2]) * np.exp(1j * pos[:, None] * 10000.0 ** (-j / 32.0))
     bad = v41.rope_tail(x, pos, theta=500000.0)
     assert not np.allclose(bad[:, 448::2], z.real, atol=1e-12)
+
+
+def _fp4_appends_match_cache_write(append):
+    r = np.random.default_rng(5)
+    lat = r.standard_normal((1, 12, 512))
+    bt = np.array([[1, 0]], np.int32)
+    pool = np.zeros((2, 64, 288), np.uint8)
+    for t in range(12):
+        pool = append(pool, bt, np.array([t + 1]), lat[:, t:t + 1], 64)
+    return np.array_equal(pool[1, :12], v41.cache_write(lat)[0])
+
+
+def test_unmutated_fp4_append_passes():
+    assert _fp4_appends_match_cache_write(v41.fp4_cache_append)
+
+
+def test_append_position_off_by_one_is_caught():
+    def bad_append(pool, block_table, seq_lens, latent_new, page_size=64, tail=64, theta=10000.0):
+        lat = np.asarray(latent_new, float)
+        B, Q, D = lat.shape
+        pos = np.asarray(seq_lens)[:, None] - Q + np.arange(Q)[None, :] + 1   # the slot's position + 1
+        ent = v41.fp4_quantize(v41.rope_tail(lat, pos.astype(float), tail, theta), D)
+        return mla.cache_append(pool, block_table, seq_lens, ent, page_size)
+    assert not _fp4_appends_match_cache_write(bad_append)
+
+
+def test_append_slot_off_by_one_is_caught(monkeypatch):
+    def bad_cache_append(pool, block_table, seq_lens, rows, page_size):
+        out = np.array(pool, copy=True)
+        r = np.asarray(rows)
+        for b in range(r.shape[0]):
+            for i in range(r.shape[1]):
+                t = int(seq_lens[b]) - r.shape[1] + i + 1          # writes one slot late
+                out[int(block_table[b][t // page_size]), t % page_size] = r[b, i]
+        return out
+    monkeypatch.setattr(mla, "cache_append", bad_cache_append)
+    assert not _fp4_appends_match_cache_write(v41.fp4_cache_append)
