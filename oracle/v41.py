@@ -23,8 +23,8 @@ Readings (also listed in the design doc):
   mantissa bits 2..0, S.1111.111 = NaN, no infinities, max 448;
 - quantiser of the cache-write step (input preparation; decode parity does
   not depend on it): scale_g = E4M3(amax_g / 6) rounded to nearest-even,
-  code = E2M1(x / scale_g) rounded to nearest-even with saturation at 6,
-  zero codes when scale_g = 0;
+  code = E2M1(x / scale_g) rounded to nearest-even with saturation at 6
+  and x's sign kept (-0 for a small negative x), zero codes when scale_g = 0;
 - RoPE on the last ``tail`` = 64 dims as interleaved pairs (D-tail+2j,
   D-tail+2j+1), j = 0..tail/2-1, angle = pos * theta^(-2j/tail), theta =
   10000; cache rows are rotated at their token position before
@@ -110,27 +110,44 @@ def e4m3_quantize(x):
 
 
 def e2m1_quantize(x):
-    """float64 -> 4-bit E2M1 code, nearest-even on the magnitude, saturating at 6."""
+    """float64 -> 4-bit E2M1 code, nearest-even on the magnitude, saturating at 6.
+
+    The sign bit is x's sign, also when the magnitude rounds to 0 (a negative
+    value below 0.25 becomes -0), as a floating-point conversion keeps it.
+    """
     x = np.asarray(x, F64)
     codes = np.arange(8)
     vals = e2m1_decode(codes)
     mag = codes[_nearest_even(np.abs(x), vals, codes)]
-    return np.where((x < 0) & (mag != 0), mag | 0x8, mag).astype(np.uint8)
+    return np.where(np.signbit(x), mag | 0x8, mag).astype(np.uint8)
 
 
-def fp4_quantize(latent, D: int = 512):
+def fp4_quantize(latent, D: int = 512, decide_in_f32: bool = False):
     """Cache-write quantiser: (..., 512) float -> (..., 288) uint8 entries.
 
     scale_g = E4M3(amax_g / 6), code = E2M1(x / scale_g); zero codes where
-    scale_g decodes to 0.
+    scale_g decodes to 0. The pages do not fix the precision of the two
+    quotients whose rounding picks the codes; ``decide_in_f32`` takes them
+    the way a float32 implementation does: the input rounded to float32, then
+    amax / 6 and x / scale_g each correctly rounded in float32 before the
+    nearest-even choice (the float64 default rounds only at the choice).
     """
     x = np.asarray(latent, F64)
+    if decide_in_f32:
+        x = x.astype(np.float32).astype(F64)
     g = x.reshape(x.shape[:-1] + (D // GROUP, GROUP))
     amax = np.abs(g).max(axis=-1)
-    sbytes = e4m3_quantize(amax / 6.0)
+    if decide_in_f32:
+        sbytes = e4m3_quantize((amax.astype(np.float32) / np.float32(6.0)).astype(F64))
+    else:
+        sbytes = e4m3_quantize(amax / 6.0)
     s = e4m3_decode(sbytes)
     safe = np.where(s > 0, s, 1.0)
-    codes = e2m1_quantize(g / safe[..., None])
+    if decide_in_f32:
+        q = (g.astype(np.float32) / safe[..., None].astype(np.float32)).astype(F64)
+    else:
+        q = g / safe[..., None]
+    codes = e2m1_quantize(q)
     codes = np.where((s > 0)[..., None], codes, 0).reshape(x.shape).astype(np.uint8)
     out = np.empty(x.shape[:-1] + (ENTRY_BYTES,), np.uint8)
     out[..., :D // 2] = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
@@ -169,18 +186,19 @@ def cache_write(latent, tail: int = 64, theta: float = 10000.0):
 
 
 def fp4_cache_append(pool, block_table, seq_lens, latent_new, page_size: int = 64, tail: int = 64,
-                     theta: float = 10000.0):
+                     theta: float = 10000.0, decide_in_f32: bool = False):
     """Shared-latent cache append into a paged pool of 288-byte entries.
 
     latent_new (B, Q, 512): the new tokens' latents; seq_lens: lengths after
     the append. Each new token's tail is rotated at its position
-    seq_lens[b] - Q + i, quantised to an FP4 entry, and written to its slot
-    (mla.cache_append's addressing): the per-token form of cache_write.
+    seq_lens[b] - Q + i, quantised to an FP4 entry (``decide_in_f32`` as in
+    fp4_quantize), and written to its slot (mla.cache_append's addressing):
+    the per-token form of cache_write.
     """
     lat = np.asarray(latent_new, F64)
     B, Q, D = lat.shape
     pos = np.asarray(seq_lens, np.int64)[:, None] - Q + np.arange(Q)[None, :]
-    ent = fp4_quantize(rope_tail(lat, pos.astype(F64), tail, theta), D)
+    ent = fp4_quantize(rope_tail(lat, pos.astype(F64), tail, theta), D, decide_in_f32)
     return _mla.cache_append(pool, block_table, seq_lens, ent, page_size)
 
 

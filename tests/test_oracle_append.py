@@ -101,3 +101,23 @@ def test_bad_page_or_length_raises():
         omla.cache_append(pool, np.array([[5]]), np.array([1]), np.zeros((1, 1, 8)), 64)
     with pytest.raises(ValueError):
         omla.cache_append(pool, np.array([[0]]), np.array([1]), np.zeros((1, 2, 8)), 64)
+
+
+def test_f32_decisions_agree_with_f64_away_from_ties():
+    # both modes choose the same codes unless a quotient lies within float32
+    # rounding of a nearest-even boundary; on N(0,1) latents that is rare
+    rng = np.random.Generator(np.random.PCG64(46))
+    lat = rng.standard_normal((4, 64, 512)).astype(np.float32).astype(np.float64)
+    a = v41.fp4_quantize(lat)
+    b = v41.fp4_quantize(lat, decide_in_f32=True)
+    assert (a != b).mean() < 1e-4
+
+
+def test_f32_decision_on_a_constructed_boundary():
+    # amax = 6 * 2^-3 * (1 + 1/16): amax/6 sits exactly between the E4M3 values
+    # 2^-3 and 2^-3 * (1 + 1/8); nearest-even picks the even mantissa (2^-3)
+    x = np.zeros((1, 512))
+    x[0, 0] = 6 * 0.125 * (1 + 1 / 16)
+    for mode in (False, True):
+        e = v41.fp4_quantize(x, decide_in_f32=mode)
+        assert v41.e4m3_decode(e[0, 256:257])[0] == 0.125

@@ -166,3 +166,8 @@ def test_sink_enters_split_merge_once():
         expect = (np.exp(lse[:, 0, h, 0])[:, None] * O[:, 0, h, 0]).sum(0) / den
         assert np.allclose(x[0, h, 0], expect, atol=1e-14)
         assert math.isclose(float(L[0, h, 0]), math.log(den), rel_tol=1e-12)
+
+
+def test_e2m1_quantize_keeps_the_sign_of_a_value_rounding_to_zero():
+    # a conversion rounds the magnitude and keeps the sign: -0.1 -> -0 (code 8)
+    assert list(v41.e2m1_quantize(np.array([-0.1, 0.1, -0.0, 0.0]))) == [8, 0, 8, 0]
