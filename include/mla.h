@@ -227,6 +227,56 @@ mla_status_t mla_combine(const mla_decode_args* a, const void* workspace,
 #define MLA_STATIC_SCRATCH_BYTES (32u << 20)
 mla_status_t mla_decode_static_scratch(const mla_decode_args* a, void* stream);
 
+/*
+ * mla_cache_append - the step before the decode: write each sequence's Q new
+ * tokens into the cache rows mla_decode reads. The neuronix DeepSeek-V3/R1
+ * page's LatentKVCachePool gives a token's latent and rope parts a slot at its
+ * position before attention runs; the openarchlab 4A page (§1, §4) stores the
+ * shared latent, its tail rotated at the token's position, as a 288-byte FP4
+ * entry.
+ *
+ *   c_kv  (B,Q,Ckv) new latent rows, src_dtype, contiguous.
+ *   k_pe  (B,Q,Dr)  new rope rows (already rotated), src_dtype, contiguous;
+ *         NULL when Dr == 0.
+ *   seq_lens (B) int32, required: the lengths AFTER the append. New token i
+ *     of sequence b is token t = seq_lens[b] - Q + i and goes to the row that
+ *     mla_decode reads for t: the same kv_cache / pe_cache, row and batch
+ *     strides, Lk, block_table, max_pages, page_size and num_pages rules.
+ *   cache_dtype == src_dtype (MLA_F32 or MLA_BF16): the rows are copied.
+ *   cache_dtype == MLA_FP4_E2M1_E4M3x16 (Ckv = 512, Dr = 0, src MLA_F32 or
+ *     MLA_BF16, row stride in BYTES, >= 288 and a multiple of 16): the
+ *     latent's last rope_tail (0 or 64) dims are rotated by +t, pairs
+ *     (448+2j, 449+2j) by angle t * rope_theta^(-2j/64) (angles in double,
+ *     results rounded to float); then each group of 16 channels gets
+ *     scale = E4M3(amax / 6) and codes E2M1(x / scale), both rounded to
+ *     nearest-even from float32 quotients with saturation (x's sign kept; a
+ *     zero scale gives zero codes), in the entry layout mla_decode reads.
+ *   err_flag: optional device int32; a token with t outside [0, Lk) or a page
+ *     id outside [0, num_pages) sets MLA_DEVICE_ERR_BLOCK_TABLE and is not
+ *     written.
+ */
+typedef struct mla_append_args {
+  int B, Q;
+  int Ckv, Dr;
+  mla_dtype_t src_dtype;   /* MLA_F32 or MLA_BF16 (c_kv, k_pe) */
+  mla_dtype_t cache_dtype; /* src_dtype, or MLA_FP4_E2M1_E4M3x16 */
+  const void* c_kv;
+  const void* k_pe;
+  void* kv_cache;
+  void* pe_cache;
+  int64_t kv_row_stride, pe_row_stride;      /* elements (bytes for FP4) */
+  int64_t kv_batch_stride, pe_batch_stride;  /* contiguous layout only */
+  int Lk;                  /* contiguous: rows per sequence; paged: max_pages*page_size */
+  const int32_t* seq_lens; /* (B), lengths after the append */
+  const int32_t* block_table; /* (B,max_pages) or NULL */
+  int max_pages, page_size, num_pages;
+  int rope_tail;           /* FP4 only: 0 or 64 */
+  float rope_theta;
+  int32_t* err_flag;       /* optional device status word */
+} mla_append_args;
+
+mla_status_t mla_cache_append(const mla_append_args* a, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,6 +7,7 @@
 
 #include <mutex>
 
+#include "append.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -301,4 +302,53 @@ extern "C" mla_status_t mla_decode_static_scratch(const mla_decode_args* a, void
   s = mla_decode(a, ws, need, stream);
   if (s != MLA_OK) return s;
   return mla_combine(a, ws, need, stream);
+}
+
+// ---------------------------------------------------------------------------
+// cache append
+// ---------------------------------------------------------------------------
+namespace {
+
+mla_status_t validate_append(const mla_append_args* a) {
+  if (!a) return MLA_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->Q <= 0 || a->Lk <= 0 || a->Ckv <= 0 || a->Dr < 0) return MLA_ERR_INVALID_ARG;
+  if (a->src_dtype != MLA_F32 && a->src_dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  const bool fp4 = a->cache_dtype == MLA_FP4_E2M1_E4M3x16;
+  if (!fp4 && a->cache_dtype != a->src_dtype) return MLA_ERR_UNSUPPORTED;
+  if (!a->c_kv || !a->kv_cache || !a->seq_lens) return MLA_ERR_INVALID_ARG;
+  if (a->Dr > 0 && (!a->k_pe || !a->pe_cache)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(a->seq_lens, 4) || (a->block_table && !aligned(a->block_table, 4)) ||
+      (a->err_flag && !aligned(a->err_flag, 4)))
+    return MLA_ERR_INVALID_ARG;
+  const int64_t esz = a->src_dtype == MLA_F32 ? 4 : 2;
+  if (!aligned(a->c_kv, esz) || (a->Dr > 0 && !aligned(a->k_pe, esz))) return MLA_ERR_INVALID_ARG;
+  if (fp4) {
+    if (a->Ckv != mla::kCkv || a->Dr != 0) return MLA_ERR_UNSUPPORTED;
+    if (a->rope_tail != 0 && a->rope_tail != 64) return MLA_ERR_UNSUPPORTED;
+    if (a->rope_tail && !(a->rope_theta > 0.f)) return MLA_ERR_INVALID_ARG;
+    // 8-byte code stores: entries start on 16-byte boundaries
+    if (!aligned(a->kv_cache, 16) || a->kv_row_stride < mla::kFp4EntryBytes || a->kv_row_stride % 16 != 0)
+      return MLA_ERR_INVALID_ARG;
+    if (!a->block_table && a->kv_batch_stride % 16 != 0) return MLA_ERR_INVALID_ARG;
+  } else {
+    if (a->rope_tail != 0) return MLA_ERR_UNSUPPORTED;   // rope rows arrive rotated
+    if (!aligned(a->kv_cache, esz) || a->kv_row_stride < a->Ckv) return MLA_ERR_INVALID_ARG;
+    if (a->Dr > 0 && (!aligned(a->pe_cache, esz) || a->pe_row_stride < a->Dr)) return MLA_ERR_INVALID_ARG;
+  }
+  if (a->block_table) {
+    if (a->page_size <= 0 || a->max_pages <= 0 || a->num_pages <= 0) return MLA_ERR_INVALID_ARG;
+    if ((int64_t)a->max_pages * a->page_size < a->Lk) return MLA_ERR_INVALID_ARG;
+  } else if (a->B > 1) {
+    if (a->kv_batch_stride < (int64_t)a->Lk * a->kv_row_stride) return MLA_ERR_INVALID_ARG;
+    if (a->Dr > 0 && a->pe_batch_stride < (int64_t)a->Lk * a->pe_row_stride) return MLA_ERR_INVALID_ARG;
+  }
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status_t mla_cache_append(const mla_append_args* a, void* stream) {
+  mla_status_t s = validate_append(a);
+  if (s != MLA_OK) return s;
+  return cuda_status(mla::launch_cache_append(a, (cudaStream_t)stream));
 }

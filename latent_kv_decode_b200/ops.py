@@ -17,6 +17,9 @@ Calls (same names as the C ABI):
 - ``mla_decode_step(q_nope, q_pe, kv_cache, pe_cache, wkv_b, softmax_scale,
   causal_mask)``: the four calls in a row with the signature of the 6547.cn
   question's ``mla_decode_step``.
+- ``mla_cache_append(c_kv, k_pe, kv_cache, pe_cache, seq_lens, ...)``: the
+  step before the decode, writing the new tokens' rows (or FP4 entries) into
+  the cache.
 """
 from __future__ import annotations
 
@@ -51,6 +54,7 @@ _SIGS = {
     "mla_decode": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "mla_combine": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "mla_decode_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
+    "mla_cache_append": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
 }
 
 
@@ -74,6 +78,22 @@ class DecodeArgs(ctypes.Structure):
         ("sinks", _c.c_void_p), ("rope_tail", _c.c_int), ("rope_theta", _c.c_float),
         ("num_splits", _c.c_int), ("x", _c.c_void_p), ("lse", _c.c_void_p),
         ("err_flag", _c.c_void_p),
+    ]
+
+
+class AppendArgs(ctypes.Structure):
+    """Mirror of ``mla_append_args`` in include/mla.h (field order and types)."""
+
+    _fields_ = [
+        ("B", _c.c_int), ("Q", _c.c_int), ("Ckv", _c.c_int), ("Dr", _c.c_int),
+        ("src_dtype", _c.c_int), ("cache_dtype", _c.c_int),
+        ("c_kv", _c.c_void_p), ("k_pe", _c.c_void_p), ("kv_cache", _c.c_void_p),
+        ("pe_cache", _c.c_void_p),
+        ("kv_row_stride", _c.c_int64), ("pe_row_stride", _c.c_int64),
+        ("kv_batch_stride", _c.c_int64), ("pe_batch_stride", _c.c_int64),
+        ("Lk", _c.c_int), ("seq_lens", _c.c_void_p), ("block_table", _c.c_void_p),
+        ("max_pages", _c.c_int), ("page_size", _c.c_int), ("num_pages", _c.c_int),
+        ("rope_tail", _c.c_int), ("rope_theta", _c.c_float), ("err_flag", _c.c_void_p),
     ]
 
 
@@ -296,3 +316,50 @@ def mla_decode_step(q_nope, q_pe, kv_cache, pe_cache, wkv_b, softmax_scale, caus
     q_lat = mla_absorb_q(q_nope, wkv_b, stream=kw.get("stream"))
     x, _ = decode(q_lat, q_pe, kv_cache, pe_cache, softmax_scale, causal_mask=causal_mask, **kw)
     return mla_up_proj(x, wkv_b, Dn, stream=kw.get("stream"))
+
+
+def make_append_args(c_kv, k_pe, kv_cache, pe_cache, seq_lens, *, block_table=None, page_size: int = 64,
+                     rope_tail: int = 0, rope_theta: float = 10000.0, err_flag=None,
+                     Lk: Optional[int] = None) -> AppendArgs:
+    """Fill an AppendArgs from tensors (no GPU work).
+
+    c_kv (B, Q, Ckv) / k_pe (B, Q, Dr) are the new tokens' rows; seq_lens
+    (B) int32 are the lengths after the append. The cache tensors follow
+    make_decode_args: (B, Lk, C) views or (num_pages, page_size, C) pools with
+    ``block_table``; a uint8 kv_cache of 288-byte rows takes FP4 entries.
+    """
+    _need_cuda(c_kv, k_pe, kv_cache, pe_cache, seq_lens, block_table, err_flag)
+    B, Q, Ckv = c_kv.shape
+    assert c_kv.is_contiguous() and seq_lens.dtype == torch.int32 and seq_lens.is_contiguous()
+    Dr = 0 if k_pe is None else k_pe.shape[-1]
+    if k_pe is not None:
+        assert k_pe.is_contiguous() and k_pe.dtype == c_kv.dtype
+    a = AppendArgs()
+    a.B, a.Q, a.Ckv, a.Dr = B, Q, Ckv, Dr
+    a.src_dtype = _qdtype(c_kv)
+    a.cache_dtype = MLA_FP4 if kv_cache.dtype == torch.uint8 else _qdtype(kv_cache)
+    a.c_kv, a.k_pe = _ptr(c_kv), _ptr(k_pe)
+    a.kv_cache, a.pe_cache = _ptr(kv_cache), _ptr(pe_cache)
+    assert kv_cache.stride(-1) == 1
+    a.kv_row_stride, a.kv_batch_stride = kv_cache.stride(1), kv_cache.stride(0)
+    if pe_cache is not None:
+        assert pe_cache.stride(-1) == 1
+        a.pe_row_stride, a.pe_batch_stride = pe_cache.stride(1), pe_cache.stride(0)
+    a.seq_lens = _ptr(seq_lens)
+    if block_table is not None:
+        assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+        a.block_table = _ptr(block_table)
+        a.max_pages, a.page_size, a.num_pages = block_table.shape[1], page_size, kv_cache.shape[0]
+        a.kv_batch_stride = a.pe_batch_stride = 0
+        a.Lk = Lk if Lk is not None else a.max_pages * page_size
+    else:
+        a.Lk = Lk if Lk is not None else kv_cache.shape[1]
+    a.rope_tail, a.rope_theta = int(rope_tail), float(rope_theta)
+    a.err_flag = _ptr(err_flag)
+    return a
+
+
+def mla_cache_append(c_kv, k_pe, kv_cache, pe_cache, seq_lens, *, stream=None, **kw) -> None:
+    """Enqueue mla_cache_append: write the new tokens into the cache in place."""
+    a = make_append_args(c_kv, k_pe, kv_cache, pe_cache, seq_lens, **kw)
+    _check(lib().mla_cache_append(ctypes.byref(a), _stream(stream)), "mla_cache_append")

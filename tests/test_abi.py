@@ -49,11 +49,12 @@ def test_status_strings(L):
     assert L.mla_version().decode().count(".") == 2
 
 
-def test_struct_layout_matches_header():
+@pytest.mark.parametrize("name,cls", [("mla_decode_args", "DecodeArgs"), ("mla_append_args", "AppendArgs")])
+def test_struct_layout_matches_header(name, cls):
     """ctypes mirror has the header's fields in the header's order."""
     from latent_kv_decode_b200 import ops
     src = open(HEADER).read()
-    body = src[src.index("typedef struct mla_decode_args {"):src.index("} mla_decode_args;")]
+    body = src[src.index(f"typedef struct {name} {{"):src.index(f"}} {name};")]
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
     fields = []
     for line in body.splitlines()[1:]:
@@ -62,7 +63,7 @@ def test_struct_layout_matches_header():
             continue
         decl = re.sub(r"^(const\s+)?[\w]+\s*\**\s*", "", line)
         fields += [f.strip().lstrip("*") for f in decl.split(",")]
-    assert fields == [f for f, _ in ops.DecodeArgs._fields_]
+    assert fields == [f for f, _ in getattr(ops, cls)._fields_]
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any use
@@ -137,3 +138,38 @@ def test_ops_fail_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ops.MlaError):
         ops.lib()
+
+
+def _append_args(**over):
+    from latent_kv_decode_b200 import ops
+    a = ops.AppendArgs()
+    a.B, a.Q, a.Ckv, a.Dr = 2, 1, 512, 64
+    a.src_dtype = a.cache_dtype = ops.MLA_BF16
+    a.c_kv = a.k_pe = a.kv_cache = a.pe_cache = a.seq_lens = FAKE
+    a.kv_row_stride, a.pe_row_stride = 512, 64
+    a.kv_batch_stride, a.pe_batch_stride = 512 * 100, 64 * 100
+    a.Lk = 100
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+_FP4 = dict(cache_dtype=2, Dr=0, k_pe=None, pe_cache=None, kv_row_stride=288, kv_batch_stride=288 * 100)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(c_kv=None), 1), (dict(kv_cache=None), 1), (dict(seq_lens=None), 1), (dict(k_pe=None), 1),
+    (dict(B=0), 1), (dict(Q=0), 1), (dict(Lk=0), 1), (dict(src_dtype=2, cache_dtype=2), 2),
+    (dict(src_dtype=0), 2),                              # float32 rows into a bf16 cache
+    (dict(rope_tail=64), 2),                             # bf16 rope rows arrive rotated
+    (dict(kv_row_stride=100), 1), (dict(kv_batch_stride=10), 1), (dict(seq_lens=FAKE + 2), 1),
+    (dict(block_table=FAKE, page_size=64, max_pages=1, num_pages=4), 1),   # 64 < Lk
+    (dict(block_table=FAKE, page_size=0, max_pages=2, num_pages=4), 1),
+    (dict(_FP4, Ckv=256), 2), (dict(_FP4, Dr=64, k_pe=FAKE, pe_cache=FAKE), 2), (dict(_FP4, rope_tail=32), 2),
+    (dict(_FP4, kv_row_stride=280), 1), (dict(_FP4, kv_row_stride=296), 1),
+    (dict(_FP4, kv_cache=FAKE + 8), 1), (dict(_FP4, kv_batch_stride=288 * 100 + 8), 1),
+    (dict(_FP4, rope_tail=64, rope_theta=0.0), 1),
+])
+def test_append_rejects_bad_arguments(L, over, status):
+    a = _append_args(**over)
+    assert L.mla_cache_append(ctypes.byref(a), None) == status
