@@ -199,7 +199,7 @@ mla_status_t mla_combine(const mla_decode_args* a, const void* workspace,
 
 /*
  * mla_decode_static_scratch - mla_decode followed by mla_combine, for callers
- * that may not allocate device memory. The paper has no counterpart: this is
+ * that may not allocate device memory. The source pages have no counterpart: this is
  * a deployment variant of the two calls above.
  *
  * Some callers cannot call cudaMalloc or take memory from an allocator: a

@@ -7,7 +7,7 @@
 //   decode_simt     scores, scale, mask, online softmax, latent aggregation
 //                   (blanks [2]-[4], step 5), FP4 entries, sinks, inverse RoPE
 //   combine_warp    log-sum-exp merge of split partials + epilogue, a warp
-//                   per row (Ckv 128 / 256 / 512, 16-byte aligned buffers)
+//                   per row (Ckv = 512, 16-byte aligned buffers)
 //   combine_simt    the same merge for any other shape
 //
 // All arithmetic is float32; inputs are float32 or bf16 (converted on load).
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(128) combine_simt(DecodeParams p) {
   if (p.lse && threadIdx.x == 0) p.lse[grow] = red[0];
 }
 
-// combine, warp per row: for Ckv = 32 * kCols. The splits' lse values are
+// combine, warp per row: Ckv = 32 * kCols. The splits' lse values are
 // reduced across lanes; lane i owns columns [kCols i, kCols i + kCols) and
 // issues all its 16-byte partial-O loads of a group of splits before using
 // them, so a row costs a few memory latencies rather than one per split.
@@ -519,11 +519,7 @@ cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, bool fp4, cudaS
 template <typename TQ>
 static cudaError_t combine_warp_launch(const DecodeParams& p, cudaStream_t st) {
   const unsigned grid = (unsigned)(((int64_t)p.B * p.HQ + 3) / 4);
-  switch (p.Ckv) {
-    case 128: combine_warp<TQ, 4><<<grid, 128, 0, st>>>(p); break;
-    case 256: combine_warp<TQ, 8><<<grid, 128, 0, st>>>(p); break;
-    default: combine_warp<TQ, 16><<<grid, 128, 0, st>>>(p); break;
-  }
+  combine_warp<TQ, kCkv / 32><<<grid, 128, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -531,7 +527,7 @@ cudaError_t launch_combine_simt(const DecodeParams& p, bool bf16, cudaStream_t s
   const int64_t rows = (int64_t)p.B * p.HQ;
   // 16-byte loads and stores: the partials and outputs are row-contiguous
   // with rows of Ckv elements, and the buffers come from the allocator
-  const bool vec = (p.Ckv == 128 || p.Ckv == 256 || p.Ckv == 512) &&
+  const bool vec = p.Ckv == kCkv &&
                    (reinterpret_cast<uintptr_t>(p.ws_o) & 15u) == 0 &&
                    (reinterpret_cast<uintptr_t>(p.x) & 15u) == 0 && (p.rope_tail & 1) == 0;
   if (vec) return bf16 ? combine_warp_launch<__nv_bfloat16>(p, st) : combine_warp_launch<float>(p, st);
