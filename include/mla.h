@@ -24,8 +24,11 @@
  * Conventions for every call:
  *  - Tensor pointers are DEVICE pointers owned by the caller. The library
  *    allocates no device memory and keeps no per-call state; calls are
- *    re-entrant. Arrays are row-major (C order) and densely packed unless a
- *    stride argument says otherwise.
+ *    re-entrant. The one piece of library-global device state is the scratch
+ *    array of mla_decode_static_scratch (a static device array, with its
+ *    address looked up once per device); no other call touches it. Arrays
+ *    are row-major (C order) and densely packed unless a stride argument says
+ *    otherwise.
  *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream) and returns without synchronising.
  *  - Arguments are validated on the host before anything is enqueued; a call
@@ -217,6 +220,9 @@ mla_status_t mla_combine(const mla_decode_args* a, const void* workspace,
  *     mla_decode_workspace_size); one split needs no scratch at all.
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process, so this entry point
+ *     does not support cudaDeviceReset (which reloads the module and moves
+ *     the array) between its calls on a device.
  *   - All calls share the one array, whatever the stream. Calls whose GPU
  *     work overlaps in time race on it and give wrong results: serialise them
  *     (one stream, or events). The array keeps the last call's contents;

@@ -174,7 +174,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA. No TMA or bulk load in this library uses cluster multicast; the only
+// .multicast::cluster operand is tcgen05.commit's mbarrier arrive to the two
+// CTAs of one pair on the same GPU (mma_commit_2sm_mc below).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

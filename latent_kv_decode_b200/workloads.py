@@ -261,6 +261,39 @@ def fp4_random_entries(B: int, Lk: int, Ckv: int = 512, seed: int = 5) -> np.nda
     return np.concatenate([codes, scales], axis=-1)
 
 
+def layout_only(name: str, seed: int) -> Workload:
+    """The named workload's shapes, lengths and page table without its large
+    arrays (q, caches, weights are None): for timing runs that draw those
+    arrays on the device. Lengths come from the workload's own first draw;
+    the page permutation is drawn right after them (the full workload draws
+    it after the arrays, so the two tables differ)."""
+    B, H, Q, Lk = {"dsv3_b64_lk4096": (64, 128, 1, 4096), "ragged_paged_b128_q2": (128, 128, 2, 0),
+                   "longctx_b4_lk131072": (4, 128, 1, 131072),
+                   "v41_fp4_sink_h64": (32, 64, 1, 8192)}[name]
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w = Workload(name=name, B=B, H=H, Q=Q, Dn=128, Dr=64, Vd=128, Ckv=512, Lk=Lk, dtype="bf16",
+                 softmax_scale=1.0 / math.sqrt(192), q_nope=None, q_pe=None, kv_cache=None,
+                 pe_cache=None, wkv_b=None)
+    if name == "ragged_paged_b128_q2":
+        w.seq_lens = rng.integers(512, 16384, size=B, endpoint=True).astype(np.int32)
+        w.Lk = int(w.seq_lens.max())
+        w.causal = True
+        npages = [(int(L) + PAGE_SIZE - 1) // PAGE_SIZE for L in w.seq_lens]
+        perm = rng.permutation(int(sum(npages))).astype(np.int32)
+        bt = np.full((B, max(npages)), -1, np.int32)
+        k = 0
+        for b in range(B):
+            bt[b, :npages[b]] = perm[k:k + npages[b]]
+            k += npages[b]
+        w.block_table = bt
+    if name == "v41_fp4_sink_h64":
+        w.Dn = w.Dr = w.Vd = 0
+        w.softmax_scale = 1.0 / math.sqrt(512)
+        w.rope_tail = 64
+        w.extra["shared_latent"] = True
+    return w
+
+
 WORKLOADS = {
     "demo_fp32": demo_fp32,
     "dsv3_b64_lk4096": dsv3,

@@ -18,7 +18,7 @@ absorbed score, q_absorbed . c_kv + q_rope . k_rope, is written out in the
 comments of ``MultiHeadLatentAttention.forward_inference`` on the neuronix
 page "DeepSeek-V3/R1 架构深度全景解析".
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
 
 - weight split: rows [0,Dn) of wkv_b are W_UK and the last Vd rows W_UV,
   Vd = wkv_b.shape[1] - Dn (the question's dimension-preparation lines);

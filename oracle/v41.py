@@ -13,7 +13,7 @@ Attention · latent K/V dùng chung, RoPE nửa sau và W_O nhóm":
   against the fp32 latent; RoPE on the tail checked by hand and undone by the
   inverse; cache bytes independent of the number of query heads.
 
-Readings (also listed in the design doc):
+Readings where the pages leave a step open:
 
 - entry layout, 288 B = 256 B of E2M1 codes + 32 E4M3 scales: byte i holds
   channel 2i in its low nibble and channel 2i+1 in its high nibble; byte
