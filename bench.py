@@ -8,7 +8,8 @@ mla_combine (when split) -> mla_up_proj, through the C ABI. The default
 workload is the DeepSeek-V3 decode shape (B=64, H=128, Q=1, Dn=128, Dr=64,
 Vd=128, Ckv=512, Lk=4096, bf16 storage, contiguous cache). Inputs are
 seeded synthetic data resident in HBM before timing; L2 is flushed (a
-256 MiB write) before every timed step, outside the step's events.
+256 MiB write, then a 256 MiB read so no dirty lines remain) before every
+timed step, outside the step's events.
 
 Reported (one JSON line from rank 0):
   value        decode tokens/s over all ranks (B*Q*N / max-over-ranks step time)
@@ -66,6 +67,26 @@ def spec_fraction(achieved: float, unit: str) -> float:
 L2_FLUSH_BYTES = 256 << 20
 
 
+class L2Flush:
+    """Evict the step's inputs from L2 before a timed step: write a 256 MiB
+    buffer (twice L2), then read a second 256 MiB buffer so that L2 ends up
+    holding clean lines. A write alone leaves L2 full of dirty lines whose
+    write-back would then compete with the timed step's reads (measured on
+    B200: a 268 MB stream took 57 us after a write-only flush, 45 us after
+    write + read)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def fill_(self, v: float):
+        import torch
+        self.w.fill_(v)
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -116,13 +137,13 @@ def workload_desc(w) -> dict:
                              f"(K = V), FP4 E2M1 with an E4M3 scale per 16 (288 B/token), sink, "
                              f"inverse RoPE on the last {w.rope_tail} dims, bf16 q and x",
                     B=w.B, H=w.H, Q=w.Q, Lk=w.Lk, Ckv=w.Ckv, cache="contiguous FP4 entries",
-                    l2="flushed before every timed step (256 MiB write)")
+                    l2="flushed before every timed step (256 MiB write, then 256 MiB read)")
     d = dict(workload=f"{w.name}: B={w.B} H={w.H} Q={w.Q} Dn={w.Dn} Dr={w.Dr} Vd={w.Vd} "
                       f"Ckv={w.Ckv} Lk={w.Lk}{' ragged paged' if w.block_table is not None else ''}"
                       f", {w.dtype} storage, fp32 accumulate",
              B=w.B, H=w.H, Q=w.Q, Lk=w.Lk, Dn=w.Dn, Dr=w.Dr, Vd=w.Vd, Ckv=w.Ckv,
              cache="paged 64-token pages" if w.block_table is not None else "contiguous",
-             l2="flushed before every timed step (256 MiB write); cache larger than L2")
+             l2="flushed before every timed step (256 MiB write, then 256 MiB read); cache larger than L2")
     return d
 
 
@@ -414,8 +435,8 @@ class StepRunner:
 
 def time_steps(runner, stream, flush, steps: int, warmup: int, dist=None, breakdown_steps: int = 100):
     """Device-timed steps: W warm-up steps, then K steps each bracketed by CUDA
-    events on the launching stream, with L2 flushed (a 256 MiB write) before
-    every step outside its events; then a separate pass with an event between
+    events on the launching stream, with L2 flushed (L2Flush) before every
+    step outside its events; then a separate pass with an event between
     every two kernels for the per-kernel times. Returns per-rank means in ms."""
     import torch
     for _ in range(warmup):
@@ -576,7 +597,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         import torch.distributed as dist
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     peaks, psrc = load_peaks()
     hbm, tflops = peaks["hbm_gbs"], peaks["bf16_tflops"]
 

@@ -2,33 +2,46 @@
 // 128): blanks [2]-[4] and step 5 of mla_decode_step (the 6547.cn MLA decode
 // question), with the absorbed score of the neuronix DeepSeek-V3/R1 page.
 //
-// One 2-CTA cluster per (128-row block, sequence, split). CTA r of the pair
-// owns query rows [64r, 64r+64) of the block; every MMA is a pair MMA
-// (tcgen05 cta_group::2, M = 128), so each SM computes its own 64 rows and the
-// pair shares one K tile. Per 128-token tile of the cache:
+// One 2-CTA cluster per (128-row block, sequence, split). Per 128-token tile
+// of the cache, CTA r loads its own 64 tokens [64r, 64r+64) once: the eight
+// 64-dim latent chunks as two 32 KB TMA boxes (chunks 0, 1, 4, 5 into slots
+// 0-3 and chunks 2, 3, 6, 7 into slots 4-7 of the tile's set) and the rope
+// chunk.
 //
-//   S  = Q . K^T   over the 576 dims in 64-dim chunks (8 latent + 1 rope).
-//                  CTA r supplies tokens [64r, 64r+64) of the tile (the N half
-//                  of B), loaded as 4 stages of 2 latent chunks + 1 rope stage.
-//   softmax        online, base 2, lazy rescale (the running max only moves
-//                  when a score exceeds it by more than 2^8).
-//   O += P . V     2 halves of 256 latent columns x 2 halves of 64 tokens.
-//                  CTA r supplies latent columns [128r, 128r+128) of each half
-//                  for all 128 tokens.
+//   S  = Q . K^T       pair MMA, M = 128 (CTA r: query rows [64r, 64r+64)),
+//                      N = the 128 tokens (each CTA supplies its 64), K = 576.
+//   softmax            online, base 2, lazy rescale (a row's running max only
+//                      moves when a score exceeds it by more than 2^8).
+//   O^T += V^T . P^T   pair MMA, M = 256 latent dims (CTA r: dims
+//                      [256n + 128r, +128) for n = 0, 1), N = the 128 query
+//                      rows (each CTA supplies its rows' P), K = the tokens.
 //
-// The latent rows are therefore read twice per tile (once as K, once as V,
-// cut differently between the pair); the V read follows the K read of the
-// same rows closely enough to hit in L2, so HBM sees each cache row once (an
-// explicit L2 prefetch ahead of the K producer measured no gain and is off,
-// kPrefetchTiles = 0). Every TMA request moves 64 rows x 2 chunks
-// (16 KB) through a 4-D view of the cache whose box lands already in the
-// 128-byte-swizzled layout the MMAs read. Scores and the output accumulator
-// live in TMEM (S double-buffered: 2 x 64 columns; O: 2 x 128 columns).
+// Accumulating O transposed puts 128 rows of the tensor datapath on every
+// SM for the aggregation (the latent dims), where O = P . V would give each
+// SM only its 64 query rows. The price: for its dims, CTA r needs the peer's
+// 64 tokens too. After S(j) is computed, the four latent chunks CTA r does
+// not aggregate are dead in its shared memory; the peer tokens' chunks of
+// CTA r's dims are loaded from L2 (the peer just brought them in from HBM)
+// into exactly those slots, which is where the pair MMA's A descriptor finds
+// "tokens of the other CTA" in both CTAs. Every cache row crosses HBM once.
 //
-// Warp roles (224 threads): warp 0 K producer (+ Q), warp 1 MMA issuer (even
-// CTA only) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane =
-// 32*(warp%4) + lane), warp 6 V producer. Every wait is bounded; a timeout sets
-// MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
+// With that slot order, slots 2n, 2n+1 hold the dims of O^T half n that CTA 0
+// aggregates and slots 4 + 2n, 5 + 2n those of CTA 1; the tokens of CTA 0
+// (the first four 16-token MMA steps of the aggregation) are read from slots
+// 0-3 in both CTAs and those of CTA 1 from slots 4-7. Each CTA's peer-token
+// data is one 32 KB box into the four slots holding the dims it does not
+// aggregate, and the aggregation is issued as two halves (slots 0-3, then
+// slots 4-7) so the next tile's first box can load as soon as the first half
+// is done. Only two tile sets fit beside Q in shared memory.
+//
+// A row's rescale factor alpha touches O^T in both CTAs (column = row), so
+// each CTA sends its rows' alpha (and whether any row needs a rescale) to the
+// peer every tile; the rescale itself is rare.
+//
+// Warp roles (224 threads): warp 0 own-token producer (+ Q), warp 1 MMA issuer
+// (even CTA) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane =
+// 32*(warp%4) + lane), warp 6 peer-token producer. Every wait is bounded; a
+// timeout sets MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -43,41 +56,41 @@ using namespace sm100;
 
 constexpr int kThreads = 224;
 constexpr int kTileT = 128;                 // tokens per tile (both CTAs)
-constexpr int kKStages = 3;                 // ring of K stages: 3 chunks of 64 dims (24 KB); a tile
-constexpr int kKStage = 24576;
-constexpr int kVStages = 4;                 // ring of V stages (16 KB): a tile
-constexpr int kStage = 16384;               // V stage bytes per CTA
-constexpr int kKUses = 3;                   // K stage uses per tile: chunks 0-2, 3-5, 6-7 + rope
-constexpr int kPrefetchTiles = 0;           // L2 prefetch distance of the K producer (off: measured no gain)
-constexpr int kQBlocks = 9;                 // 64-dim blocks of the 576-wide query row
-constexpr int kQBytes = kQBlocks * 8192;    // 64 rows x 128 B per block
-constexpr int kPBuf = 16384;                // P: 64 rows x 128 tokens bf16 (2 blocks), one buffer
+constexpr int kChunk = 8192;                // 64 rows (tokens or query rows) x 128 B
+constexpr int kQBytes = 9 * kChunk;         // q_lat chunks 0-7, q_pe
 
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kKStage;
-constexpr int kOffP = kOffV + kVStages * kStage;
-constexpr int kOffBar = kOffP + kPBuf;
+constexpr int kOffL = kOffQ + kQBytes;      // 2 sets x 8 latent chunk slots
+constexpr int kOffR = kOffL + 16 * kChunk;  // rope chunk slot
+constexpr int kOffP = kOffR + kChunk;       // P: 2 blocks (tokens 0-63, 64-127) of 64 rows x 128 B
+constexpr int kOffAux = kOffP + 2 * kChunk;
 enum : int {
-  B_KFULL = 0,
-  B_KEMPTY = B_KFULL + kKStages,
-  B_VFULL = B_KEMPTY + kKStages,
-  B_VEMPTY = B_VFULL + kVStages,
-  B_QFULL = B_VEMPTY + kVStages,
-  B_SFULL = B_QFULL + 1,
-  B_SFREE = B_SFULL + 2,
-  B_PFULL = B_SFREE + 2,
-  B_PVDONE = B_PFULL + 2,
-  B_COUNT = B_PVDONE + 2
+  B_QFULL = 0,
+  B_KF0 = 1,              // [2] latent chunks 0-3 of both CTAs landed
+  B_KF1 = 3,              // [2] latent chunks 2, 3, 6, 7 (slots 4-7) of both CTAs landed
+  B_XF = 5,               // [2] peer-token chunks of both CTAs landed
+  B_SFULL = 7,            // [2] S(j) computed (both CTAs, multicast commit)
+  B_SFREE = 9,            // [2] S buffer read by both CTAs (count 2)
+  B_PFULL = 11,           // P(j) written and O^T rescaled by both CTAs (count 2)
+  B_PVDONE = 12,          // [2] O^T += V^T P^T of tile j done (both CTAs, multicast)
+  B_AX = 14,              // [2] the peer's alpha of tile j arrived (64 + 1 asynchronous 4-byte stores)
+  B_EPX = 16,             // the peer's output scales arrived (64 asynchronous 4-byte stores)
+  B_QH0 = 17,             // [2] QK(j) over slots 0-3 done (both CTAs, multicast)
+  B_PVX = 19,             // [2] PV(j) over slots 0-3 done (both CTAs, multicast)
+  B_RF = 21,              // the rope chunk of tile j of both CTAs landed (phase j)
+  B_COUNT = 22
 };
-constexpr int kOffTmemPtr = kOffBar + B_COUNT * 8;
+constexpr int kOffTmemPtr = kOffAux + 256;
 constexpr int kOffAbort = kOffTmemPtr + 4;
-constexpr int kOffXchg = kOffBar + 512;     // float xmax[2][128], xsum[128]
-constexpr int kSmemBytes = kOffXchg + 3 * 128 * 4;
+constexpr int kOffFlags = kOffAux + 272;    // int need[2][2]
+constexpr int kOffXmax = kOffAux + 320;     // float [128]: token-half exchange
+constexpr int kOffAlpha = kOffXmax + 512;   // float [2][128]: alpha (epilogue: output scale)
+constexpr int kSmemBytes = kOffAlpha + 1024;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
+static_assert(kSmemAlloc <= 232448, "shared memory over the per-block limit");
 
-constexpr uint32_t kColS = 0;               // S buffers at columns 0 and 64
-constexpr uint32_t kColO = 128;             // O halves at columns 128 and 256
+constexpr uint32_t kColS = 0;               // S buffers at columns 0 and 64 (pair M = 128 layout)
+constexpr uint32_t kColO = 128;             // O^T halves n = 0, 1 at columns 128 and 256
 constexpr uint32_t kTmemCols = 512;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -87,8 +100,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct alignas(64) Sm100Params {
   CUtensorMap tm_q;    // q_lat  (B*HQ, 512), box 64 x 64
   CUtensorMap tm_qpe;  // q_pe   (B*HQ, 64),  box 64 x 64
-  CUtensorMap tm_k;    // latent cache as (64 dims, rows, 8 chunks, seq|page): box 64 rows x 2 chunks
-  CUtensorMap tm_k3;   // the same view, box 64 rows x 3 chunks
+  CUtensorMap tm_kx;   // latent cache as (64 dims, rows, 4 chunks, 2 groups of 4, seq|page):
+                       // box 64 rows x 2 chunks x 2 groups = chunks c, c+1, c+4, c+5
   CUtensorMap tm_pe;   // rope cache (64 dims, rows, seq|page): box 64 rows
   DecodeParams p;
   int paged;
@@ -149,25 +162,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   const uint32_t rank = cluster_ctarank();
   const int rb = blockIdx.x >> 1, b = blockIdx.y, z = blockIdx.z;
   pdl_launch_dependents();
-  auto bar = [&](int i) -> uint32_t { return sb0 + kOffBar + 8u * (uint32_t)i; };
+  auto bar = [&](int i) -> uint32_t { return sb0 + kOffAux + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_KEMPTY + s), 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
-    }
     mbar_init(bar(B_QFULL), 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_KF0 + i), 1);
+      mbar_init(bar(B_KF1 + i), 1);
+      mbar_init(bar(B_XF + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
       mbar_init(bar(B_SFREE + i), 2);   // one arrival per CTA
-      mbar_init(bar(B_PFULL + i), 2);   // one arrival per CTA
       mbar_init(bar(B_PVDONE + i), 1);
+      mbar_init(bar(B_AX + i), 1);      // local expect_tx; the peer's stores count the bytes
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_QH0 + i), 1);
+      mbar_init(bar(B_PVX + i), 1);
+    }
+    mbar_init(bar(B_RF), 1);
+    mbar_init(bar(B_PFULL), 2);         // one arrival per CTA
+    mbar_init(bar(B_EPX), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -197,23 +212,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     while (global_ns() - t0 < 50000ull) {
     }
   };
+  // TMA coordinates of the 64 tokens starting at t: (row, seq|page)
+  auto coords = [&](int t, int& y, int& zc) {
+    if (P.paged) {
+      zc = page_of(p, b, t, len);
+      y = 0;
+    } else {
+      zc = b;
+      y = t;
+    }
+  };
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ K producer
-    // Q once, then for every tile the 9 K chunks (this CTA's 64 tokens x 64 dims).
+    // ------------------------------------------------------------------ own-token producer
     if (lane == 0) {
       tma_prefetch_desc(&P.tm_q);
       tma_prefetch_desc(&P.tm_qpe);
-      tma_prefetch_desc(&P.tm_k);
-      tma_prefetch_desc(&P.tm_k3);
+      tma_prefetch_desc(&P.tm_kx);
       tma_prefetch_desc(&P.tm_pe);
       const int qrow = b * p.HQ + rb * 128 + (int)rank * 64;
       const uint32_t qbar = map_to_rank(bar(B_QFULL), 0);
       if (rank == 0) mbar_arrive_expect_tx(bar(B_QFULL), 2 * kQBytes);
-      for (int c = 0; c < 8; ++c) tma_load_2d_2sm(sb0 + kOffQ + c * 8192, &P.tm_q, qbar, 64 * c, qrow);
-      tma_load_2d_2sm(sb0 + kOffQ + 8 * 8192, &P.tm_qpe, qbar, 0, qrow);
-      // L2 prefetch of this CTA's 64 cache rows of a tile (latent and rope rows
-      // as whole contiguous ranges), kPrefetchTiles ahead of the shared-memory loads
+      for (int c = 0; c < 8; ++c) tma_load_2d_2sm(sb0 + kOffQ + c * kChunk, &P.tm_q, qbar, 64 * c, qrow);
+      tma_load_2d_2sm(sb0 + kOffQ + 8 * kChunk, &P.tm_qpe, qbar, 0, qrow);
+      // L2 prefetch of this CTA's 64 cache rows of tile jt (latent and rope rows
+      // as contiguous ranges), one tile ahead of its shared-memory load: the
+      // load in the tile-to-tile dependency chain then hits L2
       auto prefetch_tile = [&](int jt) {
         const int t = t_begin + jt * kTileT + (int)rank * 64;
         if (jt >= ntiles || t >= len) return;
@@ -228,33 +252,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
           kvb += ((int64_t)b * p.kv_batch + (int64_t)t * p.kv_row) * 2;
           peb += ((int64_t)b * p.pe_batch + (int64_t)t * p.pe_row) * 2;
         }
-        // the range ends at the last row's own data (strided rows may share a buffer)
+        // each range ends at the last row's own data (strided rows may share a buffer)
         prefetch_l2_bulk(kvb, (uint32_t)(((int64_t)(rows - 1) * p.kv_row + p.Ckv) * 2));
         prefetch_l2_bulk(peb, (uint32_t)(((int64_t)(rows - 1) * p.pe_row + p.Dr) * 2));
       };
-      for (int jt = 0; jt < kPrefetchTiles; ++jt) prefetch_tile(jt);
-      uint32_t it = 0;
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
-        if (kPrefetchTiles > 0) prefetch_tile(j + kPrefetchTiles);
-        const int t = t_begin + j * kTileT + (int)rank * 64;
-        int y = t, zc = b;
-        if (P.paged) {
-          zc = page_of(p, b, t, len);
-          y = 0;
-        }
-        for (int u = 0; u < kKUses; ++u, ++it) {
-          const uint32_t s = it % kKStages, round = it / kKStages;
-          if (round > 0 && !mbar_wait_cluster(bar(B_KEMPTY + s), (round - 1) & 1)) { ok = false; break; }
-          const uint32_t dst = sb0 + kOffK + s * kKStage, fb = map_to_rank(bar(B_KFULL + s), 0);
-          if (rank == 0) mbar_arrive_expect_tx(bar(B_KFULL + s), 2 * kKStage);
-          if (u < 2) {
-            tma_load_4d_2sm(dst, &P.tm_k3, fb, 0, y, 3 * u, zc);
-          } else {
-            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 6, zc);
-            tma_load_3d_2sm(dst + 2 * 8192, &P.tm_pe, fb, 0, y, zc);
-          }
-        }
+        const int s = j & 1;
+        prefetch_tile(j + 1);
+        // slots 0-3 of set s held tile j-2 until the first half of its aggregation
+        if (j >= 2 && !mbar_wait_cluster(bar(B_PVX + s), ((j - 2) >> 1) & 1)) { ok = false; break; }
+        int y, zc;
+        coords(t_begin + j * kTileT + (int)rank * 64, y, zc);
+        const uint32_t dst = sb0 + kOffL + s * 8 * kChunk;
+        if (rank == 0) mbar_arrive_expect_tx(bar(B_KF0 + s), 2 * 4 * kChunk);
+        tma_load_5d_2sm(dst, &P.tm_kx, map_to_rank(bar(B_KF0 + s), 0), 0, y, 0, 0, zc);
+        // slots 4-7 until the second half
+        if (j >= 2 && !mbar_wait_cluster(bar(B_PVDONE + s), ((j - 2) >> 1) & 1)) { ok = false; break; }
+        if (rank == 0) mbar_arrive_expect_tx(bar(B_KF1 + s), 2 * 4 * kChunk);
+        tma_load_5d_2sm(dst + 4 * kChunk, &P.tm_kx, map_to_rank(bar(B_KF1 + s), 0), 0, y, 2, 0, zc);
+        // the single rope slot once S(j-1) is computed (QK takes the rope chunk last)
+        if (j >= 1 && !mbar_wait_cluster(bar(B_SFULL + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
+        if (rank == 0) mbar_arrive_expect_tx(bar(B_RF), 2 * kChunk);
+        tma_load_3d_2sm(sb0 + kOffR, &P.tm_pe, map_to_rank(bar(B_RF), 0), 0, y, zc);
         if (*abort_flag) ok = false;
       }
       if (!ok) {
@@ -264,30 +284,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     }
     __syncwarp();
   } else if (warp == 6) {
-    // ------------------------------------------------------------------ V producer
-    // For tile j, after QK(j) has completed (these rows sit in L2): for each
-    // 256-column half and each 64-token half, this CTA's 128 latent columns.
+    // ------------------------------------------------------------------ peer-token producer
+    // The peer tokens' chunks of this CTA's aggregation dims (CTA 0: chunks 0,
+    // 1, 4, 5; CTA 1: 2, 3, 6, 7) go, as one box, to the four slots holding the
+    // chunks this CTA does not aggregate (CTA 0: slots 4-7, free once S(j) is
+    // computed; CTA 1: slots 0-3, free once QK(j) has passed them).
     if (lane == 0) {
-      uint32_t it = 0;
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
-        if (!mbar_wait_cluster(bar(B_SFULL + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
-        const int tj = t_begin + j * kTileT;
-        for (int n = 0; n < 2 && ok; ++n) {
-          for (int th = 0; th < 2; ++th, ++it) {
-            const int t = tj + 64 * th;
-            int y = t, zc = b;
-            if (P.paged) {
-              zc = page_of(p, b, t, len);
-              y = 0;
-            }
-            const uint32_t s = it % kVStages, round = it / kVStages;
-            if (round > 0 && !mbar_wait_cluster(bar(B_VEMPTY + s), (round - 1) & 1)) { ok = false; break; }
-            if (rank == 0) mbar_arrive_expect_tx(bar(B_VFULL + s), 2 * kStage);
-            const uint32_t dst = sb0 + kOffV + s * kStage, fb = map_to_rank(bar(B_VFULL + s), 0);
-            tma_load_4d_2sm(dst, &P.tm_k, fb, 0, y, 4 * n + 2 * (int)rank, zc);
-          }
-        }
+        const int s = j & 1;
+        if (!mbar_wait_cluster(bar((rank == 0 ? B_SFULL : B_QH0) + s), (j >> 1) & 1)) { ok = false; break; }
+        int y, zc;
+        coords(t_begin + j * kTileT + (1 - (int)rank) * 64, y, zc);
+        if (rank == 0) mbar_arrive_expect_tx(bar(B_XF + s), 2 * 4 * kChunk);
+        tma_load_5d_2sm(sb0 + kOffL + (s * 8 + 4 * (1 - (int)rank)) * kChunk, &P.tm_kx,
+                        map_to_rank(bar(B_XF + s), 0), 0, y, 2 * (int)rank, 0, zc);
         if (*abort_flag) ok = false;
       }
       if (!ok) {
@@ -298,72 +309,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
-    // Two independent streams, polled: QK(j) (needs S(j-2) released and K
-    // stages) and PV(j) (needs P(j) and V stages). Neither waits on the other,
-    // so a V stage in flight never stalls the K ring and vice versa.
+    // Two streams, polled: PV(j) once P(j) and the peer tokens are in (first:
+    // it frees tile j's slots), and QK(j) in two halves (chunks 0-3 as soon
+    // as they land, then chunks 4-7 + rope); a PV goes between QK halves as
+    // soon as it is ready.
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint32_t idesc_pv = idesc_bf16_f32(256, 128, true, false);
       const uint64_t qd0 = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
-      const uint64_t kd0 = smem_desc(sb0 + kOffK, 16, 1024, kSwizzle128B);
+      const uint64_t kd0 = smem_desc(sb0 + kOffL, 16, 1024, kSwizzle128B);
+      const uint64_t rd0 = smem_desc(sb0 + kOffR, 16, 1024, kSwizzle128B);
+      const uint64_t vd0 = smem_desc(sb0 + kOffL, kChunk, 1024, kSwizzle128B);
       const uint64_t pd0 = smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
-      const uint64_t vd0 = smem_desc(sb0 + kOffV, 8192, 1024, kSwizzle128B);
       bool ok = mbar_wait_cluster(bar(B_QFULL), 0);
-      uint32_t kit = 0, vit = 0;
-      int qj = 0, qu = 0;   // next QK: tile, stage use (4 latent pairs + rope)
-      int pj = 0, pu = 0;   // next PV: tile, stage use (n * 2 + token half)
+      int qj = 0, qh = 0;   // next QK: tile, half
+      int pj = 0;           // next PV: tile
       uint64_t t_idle = global_ns();
       uint32_t idle = 0;
       while (ok && pj < ntiles) {
         bool prog = false;
-        if (qj < ntiles) {
-          const int sbuf = qj & 1;
-          const bool sfree = qu > 0 || qj < 2 || mbar_poll_cluster(bar(B_SFREE + sbuf), ((qj - 2) >> 1) & 1);
-          const uint32_t s = kit % kKStages;
-          if (sfree && mbar_poll_cluster(bar(B_KFULL + s), (kit / kKStages) & 1)) {
+        if (pj < qj) {
+          const int s = pj & 1;
+          if (mbar_poll_cluster(bar(B_PFULL), pj & 1) && mbar_poll_cluster(bar(B_XF + s), (pj >> 1) & 1)) {
             tc_fence_after();
-            const uint32_t d = tmem + kColS + 64u * sbuf;
-            // Q's 64-dim blocks 3 qu .. 3 qu + 2 (block 8 = rope) against the stage's three
-            const uint64_t qd = desc_advance(qd0, 3 * qu * 8192);
-            const uint64_t kd = desc_advance(kd0, s * kKStage);
+            // first half: the tokens of CTA 0 (slots 2n, 2n+1), then the tokens of
+            // CTA 1 (slots 4+2n, 5+2n); A = V^T, 128 dims of half n; B = P^T
 #pragma unroll
-            for (int cc = 0; cc < 3; ++cc) {
+            for (int hv = 0; hv < 2; ++hv) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                mma_bf16_ss_2sm(d, desc_advance(qd, cc * 8192 + 32 * k), desc_advance(kd, cc * 8192 + 32 * k),
-                                idesc_qk, (qu | cc | k) != 0);
+              for (int n = 0; n < 2; ++n) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const int k = 4 * hv + kk;
+                  const uint64_t vd = desc_advance(vd0, (s * 8 + 4 * hv + 2 * n) * kChunk + kk * 2048);
+                  const uint64_t pd = desc_advance(pd0, hv * kChunk + kk * 32);
+                  mma_bf16_ss_2sm(tmem + kColO + 128u * n, vd, pd, idesc_pv, (pj > 0 || k > 0) ? 1u : 0u);
+                }
               }
+              mma_commit_2sm_mc(bar((hv == 0 ? B_PVX : B_PVDONE) + s), 3);
             }
-            mma_commit_2sm_mc(bar(B_KEMPTY + s), 3);
-            ++kit;
-            if (++qu == kKUses) {
-              mma_commit_2sm_mc(bar(B_SFULL + sbuf), 3);
-              qu = 0;
-              ++qj;
-            }
+            ++pj;
             prog = true;
           }
         }
-        if (pj < qj) {
-          const bool pready = pu > 0 || mbar_poll_cluster(bar(B_PFULL + (pj & 1)), (pj >> 1) & 1);
-          const uint32_t s = vit % kVStages;
-          if (pready && mbar_poll_cluster(bar(B_VFULL + s), (vit / kVStages) & 1)) {
+        if (qj < ntiles) {
+          // QK(j) in three groups: slots 0-3, slots 4-7, the rope chunk
+          const int s = qj & 1;
+          const bool sfree = qh > 0 || qj < 2 || mbar_poll_cluster(bar(B_SFREE + s), ((qj - 2) >> 1) & 1);
+          const bool ready = qh == 2 ? mbar_poll_cluster(bar(B_RF), qj & 1)
+                                     : mbar_poll_cluster(bar((qh == 0 ? B_KF0 : B_KF1) + s), (qj >> 1) & 1);
+          if (sfree && ready) {
             tc_fence_after();
-            const int n = pu >> 1, th = pu & 1;
-            const uint64_t pd = desc_advance(pd0, th * 8192);
-            const uint64_t vd = desc_advance(vd0, s * kStage);
+            const uint32_t d = tmem + kColS + 64u * s;
+            const int nc = qh == 2 ? 1 : 4;
+#pragma unroll 1
+            for (int cc = 0; cc < nc; ++cc) {
+              // slot 4 qh + cc holds latent chunk (0, 1, 4, 5, 2, 3, 6, 7)[slot]; then the rope
+              const int slot = 4 * qh + cc;
+              const int c = qh == 2 ? 8 : ((slot & 2) << 1) | ((slot & 4) >> 1) | (slot & 1);
+              const uint64_t qd = desc_advance(qd0, c * kChunk);
+              const uint64_t kd = qh == 2 ? rd0 : desc_advance(kd0, (s * 8 + slot) * kChunk);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              // P: K-block th (64 tokens), 16 tokens per step; V: 2 blocks of 64 columns
-              mma_bf16_ss_2sm(tmem + kColO + 128u * n, desc_advance(pd, 32 * k), desc_advance(vd, 2048 * k),
-                              idesc_pv, (pj > 0 || th > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ss_2sm(d, desc_advance(qd, 32 * k), desc_advance(kd, 32 * k), idesc_qk,
+                                (qh | cc | k) != 0);
             }
-            mma_commit_2sm_mc(bar(B_VEMPTY + s), 3);
-            ++vit;
-            if (++pu == 4) {
-              mma_commit_2sm_mc(bar(B_PVDONE + (pj & 1)), 3);
-              pu = 0;
-              ++pj;
+            if (qh == 2) {
+              mma_commit_2sm_mc(bar(B_SFULL + s), 3);
+              qh = 0;
+              ++qj;
+            } else {
+              if (qh == 0) mma_commit_2sm_mc(bar(B_QH0 + s), 3);
+              ++qh;
             }
             prog = true;
           }
@@ -382,13 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     // ------------------------------------------------------------------ softmax + epilogue
     const int g = warp & 3;
     const int L = 32 * g + lane;                // TMEM lane
-    const int half = L >> 6, row = L & 63;
+    const int half = L >> 6, row = L & 63;      // S: this CTA's query row, token half
+    const bool owner = half == 0;               // one thread per query row sends its stats
     const int r = rb * 128 + (int)rank * 64 + row;
     const int q = r % p.Q;
     const int h = r / p.Q;
     const uint32_t lane_base = (uint32_t)(32 * g) << 16;
-    float* xmax = reinterpret_cast<float*>(smem + kOffXchg);
-    float* xsum = xmax + 256;
+    float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
+    float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
+    int* need_s = reinterpret_cast<int*>(smem + kOffFlags);
+    const uint32_t peer = rank ^ 1u;
     float m_run = -INFINITY, l_part = 0.f;
     bool ab = false;
     // loop-invariant parameters, read once into registers
@@ -402,6 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     for (int j = 0; j < ntiles; ++j) {
       const int sbuf = j & 1;
       float s[64];
+      // this tile's alpha exchange: 64 rescale factors and one flag from the peer
+      if (leader_thread) mbar_arrive_expect_tx(bar(B_AX + (j & 1)), 65 * 4);
       if (!ab) ab = !mbar_wait_cluster(bar(B_SFULL + sbuf), (j >> 1) & 1);
       ab = __any_sync(0xffffffffu, ab);
       if (!ab) {
@@ -424,12 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       if (causal) lim = min(lim, causal_last - tb + 1);
       if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;
       if (ab) lim = 0;
-      float mx = -INFINITY;
+      // four independent max chains (one warp per SM sub-partition: latency, not
+      // throughput, sets the pace)
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (mask == nullptr) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           s[c] = (c < lim) ? s[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
         }
       } else {
         // the question's mask, one byte per lane (tb is the same across the warp)
@@ -439,87 +463,99 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         for (int c = 0; c < 64; ++c) {
           const bool vis = c < lim && (((c < 32 ? m0 : m1) >> (c & 31)) & 1u);
           s[c] = vis ? s[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
         }
       }
-      xmax[sbuf * 128 + L] = mx;
+      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      xmax[L] = mx;
       // all four warps have read S(j) by now: release the buffer to the MMA
+      // (the arrival publishes no data; tcgen05.wait::ld already returned)
       const bool stop = bar_or(1, 128, ab);
-      if (leader_thread) mbar_arrive_remote(map_to_rank(bar(B_SFREE + sbuf), 0));
+      if (leader_thread) mbar_arrive_remote_relaxed(map_to_rank(bar(B_SFREE + sbuf), 0));
       if (stop) {
         ab = true;
         break;
       }
-      mx = fmaxf(mx, xmax[sbuf * 128 + (L ^ 64)]);
+      mx = fmaxf(mx, xmax[L ^ 64]);
       const float m_new = fmaxf(m_run, mx);
-      const bool need = (m_new - m_run) > kRescaleThreshold;
+      // the first visible score sets the reference (O^T is still zero then)
+      const bool need = m_run != -INFINITY && (m_new - m_run) > kRescaleThreshold;
       float alpha = 1.f;
-      if (need) {
-        alpha = exp2f(m_run - m_new);
-        m_run = m_new;
-      }
+      if (need) alpha = exp2f(m_run - m_new);
+      if (need || m_run == -INFINITY) m_run = m_new;
       uint32_t pk[32];
-      float psum = 0.f;
+      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
       const bool none = (m_run == -INFINITY);
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const float p0 = none ? 0.f : fast_exp2(s[2 * c] - m_run);
         const float p1 = none ? 0.f : fast_exp2(s[2 * c + 1] - m_run);
-        psum += p0 + p1;
+        ps4[c & 3] += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
-      l_part = l_part * alpha + psum;
+      l_part = l_part * alpha + ((ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
 
-      // the P buffer (and O) are free once PV(j-1) is done
+      // this CTA's rows' alpha to both CTAs (O^T column = query row)
+      const int abuf = j & 1;
+      const int col = (int)rank * 64 + row;
+      const uint32_t peer_ax = map_to_rank(bar(B_AX + abuf), peer);
+      if (owner) {
+        alpha_s[abuf * 128 + col] = alpha;
+        st_async_b32(map_to_rank(smem_u32(alpha_s + abuf * 128 + col), peer), __float_as_uint(alpha), peer_ax);
+      }
+      const bool need_cta = bar_or(1, 128, owner && need);
+      if (leader_thread) {
+        st_async_b32(map_to_rank(smem_u32(need_s + abuf * 2 + (int)rank), peer), need_cta ? 1u : 0u, peer_ax);
+      }
+
+      // the P buffer (and O^T) are free once PV(j-1) is done
       if (j >= 1 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
-      uint8_t* prow = smem + kOffP + half * 8192 + row * 128;
+      if (!ab) ab = !mbar_wait_cluster(bar(B_AX + abuf), (j >> 1) & 1);
+      ab = __any_sync(0xffffffffu, ab);
+      uint8_t* prow = smem + kOffP + half * kChunk + row * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 val = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         *reinterpret_cast<uint4*>(prow + 16 * (c ^ (row & 7))) = val;
       }
-      // rescale this lane's O row when its running max moved (PV(j-1) must be done)
-      const bool warp_need = __any_sync(0xffffffffu, need && j > 0);
-      if (warp_need) {
-        ab = __any_sync(0xffffffffu, ab);
-        if (!ab) {
-          tc_fence_after();
-          // 256 columns in 4 rounds of 64: four loads per wait
+      // rescale O^T columns whose row's running max moved (either CTA's rows)
+      const bool rescale = !ab && j > 0 && (need_cta || need_s[abuf * 2 + (int)peer] != 0);
+      if (rescale) {
+        tc_fence_after();
+        const float* al = alpha_s + abuf * 128;
 #pragma unroll 1
-          for (int c = 0; c < 16; c += 4) {
-            uint32_t v[4][16];
-            const uint32_t ta = tmem + lane_base + kColO + 16u * c;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) tmem_ld16(ta + 16u * k, v[k]);
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t v[2][16];
+            const uint32_t ta = tmem + lane_base + kColO + 128u * n + (uint32_t)c;
+            tmem_ld16(ta, v[0]);
+            tmem_ld16(ta + 16u, v[1]);
             tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 2; ++k) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[k][i] = __float_as_uint(__uint_as_float(v[k][i]) * alpha);
+              for (int i = 0; i < 16; ++i)
+                v[k][i] = __float_as_uint(__uint_as_float(v[k][i]) * al[c + 16 * k + i]);
               tmem_st16(ta + 16u * k, v[k]);
             }
           }
-          tmem_wait_st();
         }
+        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
       // P(j) of all four warps is written: one arrival for this CTA
       named_bar_sync(2, 128);
-      if (leader_thread) mbar_arrive_remote(map_to_rank(bar(B_PFULL + sbuf), 0));
+      if (leader_thread) mbar_arrive_remote_cta(map_to_rank(bar(B_PFULL), 0));
     }
 
     // ---------------------------------------------------------------- epilogue
-    xsum[L] = l_part;
+    // row statistics: both token halves, then each row's output scale to both CTAs
     ab = bar_or(1, 128, ab);
-    const float l_tot = l_part + xsum[L ^ 64];
-    if (ntiles > 0 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1);
-    ab = __any_sync(0xffffffffu, ab);
-    if (ab) fail();
-    tc_fence_after();
-    const bool have_o = ntiles > 0 && !ab;
-    const int64_t grow = (int64_t)b * p.HQ + r;
-
+    xmax[L] = l_part;
+    named_bar_sync(2, 128);
+    const float l_tot = l_part + xmax[L ^ 64];
     float scale_o, lse;
     if (p.num_splits > 1) {
       scale_o = l_tot > 0.f ? 1.f / l_tot : 0.f;
@@ -536,13 +572,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       scale_o = lfin > 0.f ? w / lfin : 0.f;
       lse = lfin > 0.f ? (mfin + log2f(lfin)) * kLn2 : -INFINITY;
     }
+    // every row's output scale, in O^T column order, to both CTAs: into the
+    // alpha buffer the last tile did not use (the peer may still be reading
+    // that one for its last rescale)
+    float* scl = alpha_s + (ntiles & 1) * 128;
+    if (leader_thread) mbar_arrive_expect_tx(bar(B_EPX), 64 * 4);
+    if (owner) {
+      const int col = (int)rank * 64 + row;
+      scl[col] = scale_o;
+      st_async_b32(map_to_rank(smem_u32(scl + col), peer), __float_as_uint(scale_o),
+                   map_to_rank(bar(B_EPX), peer));
+    }
+    const int64_t grow = (int64_t)b * p.HQ + r;
+    if (owner) {
+      if (p.num_splits > 1)
+        p.ws_lse[(int64_t)z * p.B * p.HQ + grow] = lse;
+      else if (p.lse)
+        p.lse[grow] = lse;
+    }
+    if (ntiles > 0 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1);
+    if (!ab) ab = !mbar_wait_cluster(bar(B_EPX), 0);
+    ab = __any_sync(0xffffffffu, ab);
+    ab = bar_or(1, 128, ab);
+    if (ab) fail();
+    tc_fence_after();
+    const bool have_o = ntiles > 0 && !ab;
+    // this thread's O^T lane is latent dim d of half n; its 128 columns are the
+    // block's rows. Each warp (32 dims) moves 16 rows at a time through shared
+    // memory (the free tile slots) so the output goes out as 16-byte stores of
+    // whole 64- or 128-byte row pieces.
+    const int64_t row0 = (int64_t)b * p.HQ + rb * 128;
+    // inverse RoPE of the tail: dims (D - tail + 2i, D - tail + 2i + 1) sit in
+    // lanes (L, L ^ 1); the rotation angle depends on the query index only
+    const int tail0 = p.Ckv - p.rope_tail;
+    const bool split = p.num_splits > 1;
+    uint8_t* stage = smem + kOffL + g * 2048;   // 16 rows x 32 dims x 4 B per warp
 #pragma unroll 1
     for (int n = 0; n < 2; ++n) {
+      const int d0 = 256 * n + 128 * (int)rank + 32 * g;   // this warp's first dim
+      const int d = d0 + lane;
+      const bool rot = !split && p.rope_tail > 0 && d0 + 31 >= tail0;
+      // cos / sin of the rotation for query index 0..3 (Q <= 4)
+      float c0v = 1.f, c1v = 1.f, c2v = 1.f, c3v = 1.f, s0v = 0.f, s1v = 0.f, s2v = 0.f, s3v = 0.f;
+      if (rot && d >= tail0) {
+        const double freq = pow((double)p.rope_theta, -2.0 * (double)((d - tail0) >> 1) / (double)p.rope_tail);
+        double sd, cd;
+        sincos(-(double)(len - p.Q) * freq, &sd, &cd);
+        c0v = (float)cd;
+        s0v = (float)sd;
+        if (p.Q > 1) {
+          sincos(-(double)(len - p.Q + 1) * freq, &sd, &cd);
+          c1v = (float)cd;
+          s1v = (float)sd;
+        }
+        if (p.Q > 2) {
+          sincos(-(double)(len - p.Q + 2) * freq, &sd, &cd);
+          c2v = (float)cd;
+          s2v = (float)sd;
+        }
+        if (p.Q > 3) {
+          sincos(-(double)(len - p.Q + 3) * freq, &sd, &cd);
+          c3v = (float)cd;
+          s3v = (float)sd;
+        }
+      }
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c0 = 0; c0 < 128; c0 += 16) {
         uint32_t v[16];
         if (have_o) {
-          tmem_ld16(tmem + lane_base + kColO + 128u * n + 16u * c, v);
+          tmem_ld16(tmem + lane_base + kColO + 128u * n + (uint32_t)c0, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -550,36 +648,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         }
         float f[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * scale_o;
-        const int col = 256 * n + 128 * half + 16 * c;
-        if (p.num_splits > 1) {
-          float* o = p.ws_o + ((int64_t)z * p.B * p.HQ + grow) * p.Ckv + col;
+        for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * scl[c0 + i];
+        if (rot) {
+          // the partner lane holds the other element of the pair
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(o + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
-        } else {
-          if (p.rope_tail > 0 && col >= p.Ckv - p.rope_tail) {
-            const int pos = len - p.Q + q;
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              const int jp = (col + i - (p.Ckv - p.rope_tail)) >> 1;
-              inverse_rope_pair(f[i], f[i + 1], jp, p.rope_tail, p.rope_theta, pos);
+          for (int i = 0; i < 16; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, f[i], 1);
+            if (d >= tail0) {
+              const int qq = (rb * 128 + c0 + i) % p.Q;
+              const float cc = qq == 0 ? c0v : qq == 1 ? c1v : qq == 2 ? c2v : c3v;
+              const float ss = qq == 0 ? s0v : qq == 1 ? s1v : qq == 2 ? s2v : s3v;
+              f[i] = (L & 1) ? (o * ss + f[i] * cc) : (f[i] * cc - o * ss);
             }
           }
-          uint32_t w4[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) w4[i] = pack_bf16(f[2 * i], f[2 * i + 1]);
-          uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.x) + grow * p.Ckv + col);
-          o[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          o[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
         }
+        if (split) {
+          // fp32 partials: [16 rows][32 dims] = 128 B per row, 4 x 16 B per lane
+          float* st = reinterpret_cast<float*>(stage);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) st[i * 32 + lane] = f[i];
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = (lane >> 3) + 4 * k, ch = lane & 7;
+            const uint4 val = *reinterpret_cast<const uint4*>(st + rr * 32 + 4 * ch);
+            *reinterpret_cast<uint4*>(p.ws_o + ((int64_t)z * p.B * p.HQ + row0 + c0 + rr) * p.Ckv + d0 + 4 * ch) = val;
+          }
+        } else {
+          // bf16 output: [16 rows][32 dims] = 64 B per row, 2 x 16 B per lane
+          __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stage);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) st[i * 32 + lane] = __float2bfloat16_rn(f[i]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int rr = (lane >> 2) + 8 * k, ch = lane & 3;
+            const uint4 val = *reinterpret_cast<const uint4*>(st + rr * 32 + 8 * ch);
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.x) + (row0 + c0 + rr) * p.Ckv + d0 + 8 * ch) = val;
+          }
+        }
+        __syncwarp();
       }
-    }
-    if (half == 0) {
-      if (p.num_splits > 1)
-        p.ws_lse[(int64_t)z * p.B * p.HQ + grow] = lse;
-      else if (p.lse)
-        p.lse[grow] = lse;
     }
   }
 
@@ -613,7 +722,7 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
                  const uint64_t* strides_bytes, const uint32_t* box) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint32_t elem[4] = {1, 1, 1, 1};
+  cuuint32_t elem[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
                   reinterpret_cast<const cuuint64_t*>(dims),
                   reinterpret_cast<const cuuint64_t*>(strides_bytes),
@@ -678,13 +787,13 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a,
     pe_outer_stride = (uint64_t)a->Lk * a->pe_row_stride * 2;
   }
   {
-    // (64 dims, rows, 8 chunks of 64 dims, seq|page): a box of 64 rows x 2 chunks
-    // lands as [chunk][row][128 B], two K-major (or MN-major) SW128 blocks
-    uint64_t d[4] = {64, rows_per, 8, outer};
-    uint64_t s[3] = {(uint64_t)a->kv_row_stride * 2, 128, kv_outer_stride};
-    uint32_t bk[4] = {64, 64, 2, 1}, bk3[4] = {64, 64, 3, 1};
-    if (!encode_bf16(&P.tm_k, a->kv_cache, 4, d, s, bk)) return cudaErrorInvalidValue;
-    if (!encode_bf16(&P.tm_k3, a->kv_cache, 4, d, s, bk3)) return cudaErrorInvalidValue;
+    // (64 dims, rows, 4 chunks, 2 groups of 4 chunks, seq|page): a box of 64 rows
+    // x 2 chunks x 2 groups lands as four K-major SW128 blocks of 8 KB, chunks
+    // (c, c+1, c+4, c+5) for a start chunk c of 0 or 2
+    uint64_t d[5] = {64, rows_per, 4, 2, outer};
+    uint64_t s[4] = {(uint64_t)a->kv_row_stride * 2, 128, 512, kv_outer_stride};
+    uint32_t bx[5] = {64, 64, 2, 2, 1};
+    if (!encode_bf16(&P.tm_kx, a->kv_cache, 5, d, s, bx)) return cudaErrorInvalidValue;
   }
   {
     uint64_t d[3] = {64, rows_per, outer};
