@@ -38,10 +38,13 @@
 // each CTA sends its rows' alpha (and whether any row needs a rescale) to the
 // peer every tile; the rescale itself is rare.
 //
-// Warp roles (224 threads): warp 0 own-token producer (+ Q), warp 1 MMA issuer
+// Warp roles (256 threads): warp 0 own-token producer (+ Q), warp 1 QK issuer
 // (even CTA) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane =
-// 32*(warp%4) + lane), warp 6 peer-token producer. Every wait is bounded; a
-// timeout sets MLA_DEVICE_ERR_TIMEOUT and the kernel unwinds.
+// 32*(warp%4) + lane), warp 6 peer-token producer, warp 7 PV issuer (even
+// CTA). The two issuers write disjoint TMEM (S and O^T) and each commit
+// tracks only its own thread's MMAs, so neither stream waits on the other's
+// barriers. Every wait is bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and
+// the kernel unwinds.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -54,7 +57,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr int kTileT = 128;                 // tokens per tile (both CTAs)
 constexpr int kChunk = 8192;                // 64 rows (tokens or query rows) x 128 B
 constexpr int kQBytes = 9 * kChunk;         // q_lat chunks 0-7, q_pe
@@ -308,89 +311,77 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer (even CTA)
-    // Two streams, polled: PV(j) once P(j) and the peer tokens are in (first:
-    // it frees tile j's slots), and QK(j) in two halves (chunks 0-3 as soon
-    // as they land, then chunks 4-7 + rope); a PV goes between QK halves as
-    // soon as it is ready.
+    // ------------------------------------------------------------------ QK issuer (even CTA)
+    // S(j) = Q . K^T in three groups as their data lands: slots 0-3 (then a
+    // commit that frees them for the peer-token box of CTA 1), slots 4-7, the
+    // rope chunk; the S buffer must have been read by softmax(j-2).
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(256, 128, true, false);
       const uint64_t qd0 = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
       const uint64_t kd0 = smem_desc(sb0 + kOffL, 16, 1024, kSwizzle128B);
       const uint64_t rd0 = smem_desc(sb0 + kOffR, 16, 1024, kSwizzle128B);
+      bool ok = mbar_wait_cluster(bar(B_QFULL), 0);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int s = j & 1;
+        const uint32_t d = tmem + kColS + 64u * s;
+        if (j >= 2) ok = mbar_wait_cluster(bar(B_SFREE + s), ((j - 2) >> 1) & 1);
+#pragma unroll 1
+        for (int g3 = 0; g3 < 3 && ok; ++g3) {
+          ok = g3 == 2 ? mbar_wait_cluster(bar(B_RF), j & 1)
+                       : mbar_wait_cluster(bar((g3 == 0 ? B_KF0 : B_KF1) + s), (j >> 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const int nc = g3 == 2 ? 1 : 4;
+#pragma unroll 1
+          for (int cc = 0; cc < nc; ++cc) {
+            // slot 4 g3 + cc holds latent chunk (0, 1, 4, 5, 2, 3, 6, 7)[slot]; then the rope
+            const int slot = 4 * g3 + cc;
+            const int c = g3 == 2 ? 8 : ((slot & 2) << 1) | ((slot & 4) >> 1) | (slot & 1);
+            const uint64_t qd = desc_advance(qd0, c * kChunk);
+            const uint64_t kd = g3 == 2 ? rd0 : desc_advance(kd0, (s * 8 + slot) * kChunk);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ss_2sm(d, desc_advance(qd, 32 * k), desc_advance(kd, 32 * k), idesc_qk,
+                              (g3 | cc | k) != 0);
+          }
+          if (g3 == 0) mma_commit_2sm_mc(bar(B_QH0 + s), 3);
+        }
+        if (ok) mma_commit_2sm_mc(bar(B_SFULL + s), 3);
+        if (*abort_flag) ok = false;
+      }
+      if (!ok) fail();
+    }
+    __syncwarp();
+  } else if (warp == 7) {
+    // ------------------------------------------------------------------ PV issuer (even CTA)
+    // O^T += V^T . P^T once P(j) is written by both CTAs and the peer tokens
+    // are in: first the tokens of CTA 0 (slots 2n, 2n+1 for O^T half n), a
+    // commit that frees slots 0-3, then the tokens of CTA 1 (slots 4+2n, 5+2n).
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16_f32(256, 128, true, false);
       const uint64_t vd0 = smem_desc(sb0 + kOffL, kChunk, 1024, kSwizzle128B);
       const uint64_t pd0 = smem_desc(sb0 + kOffP, 16, 1024, kSwizzle128B);
-      bool ok = mbar_wait_cluster(bar(B_QFULL), 0);
-      int qj = 0, qh = 0;   // next QK: tile, half
-      int pj = 0;           // next PV: tile
-      uint64_t t_idle = global_ns();
-      uint32_t idle = 0;
-      while (ok && pj < ntiles) {
-        bool prog = false;
-        if (pj < qj) {
-          const int s = pj & 1;
-          if (mbar_poll_cluster(bar(B_PFULL), pj & 1) && mbar_poll_cluster(bar(B_XF + s), (pj >> 1) & 1)) {
-            tc_fence_after();
-            // first half: the tokens of CTA 0 (slots 2n, 2n+1), then the tokens of
-            // CTA 1 (slots 4+2n, 5+2n); A = V^T, 128 dims of half n; B = P^T
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int s = j & 1;
+        ok = mbar_wait_cluster(bar(B_PFULL), j & 1) && mbar_wait_cluster(bar(B_XF + s), (j >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
+        for (int hv = 0; hv < 2; ++hv) {
 #pragma unroll
-              for (int n = 0; n < 2; ++n) {
+          for (int n = 0; n < 2; ++n) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const int k = 4 * hv + kk;
-                  const uint64_t vd = desc_advance(vd0, (s * 8 + 4 * hv + 2 * n) * kChunk + kk * 2048);
-                  const uint64_t pd = desc_advance(pd0, hv * kChunk + kk * 32);
-                  mma_bf16_ss_2sm(tmem + kColO + 128u * n, vd, pd, idesc_pv, (pj > 0 || k > 0) ? 1u : 0u);
-                }
-              }
-              mma_commit_2sm_mc(bar((hv == 0 ? B_PVX : B_PVDONE) + s), 3);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t vd = desc_advance(vd0, (s * 8 + 4 * hv + 2 * n) * kChunk + kk * 2048);
+              const uint64_t pd = desc_advance(pd0, hv * kChunk + kk * 32);
+              mma_bf16_ss_2sm(tmem + kColO + 128u * n, vd, pd, idesc_pv,
+                              (j > 0 || hv > 0 || kk > 0) ? 1u : 0u);
             }
-            ++pj;
-            prog = true;
           }
+          mma_commit_2sm_mc(bar((hv == 0 ? B_PVX : B_PVDONE) + s), 3);
         }
-        if (qj < ntiles) {
-          // QK(j) in three groups: slots 0-3, slots 4-7, the rope chunk
-          const int s = qj & 1;
-          const bool sfree = qh > 0 || qj < 2 || mbar_poll_cluster(bar(B_SFREE + s), ((qj - 2) >> 1) & 1);
-          const bool ready = qh == 2 ? mbar_poll_cluster(bar(B_RF), qj & 1)
-                                     : mbar_poll_cluster(bar((qh == 0 ? B_KF0 : B_KF1) + s), (qj >> 1) & 1);
-          if (sfree && ready) {
-            tc_fence_after();
-            const uint32_t d = tmem + kColS + 64u * s;
-            const int nc = qh == 2 ? 1 : 4;
-#pragma unroll 1
-            for (int cc = 0; cc < nc; ++cc) {
-              // slot 4 qh + cc holds latent chunk (0, 1, 4, 5, 2, 3, 6, 7)[slot]; then the rope
-              const int slot = 4 * qh + cc;
-              const int c = qh == 2 ? 8 : ((slot & 2) << 1) | ((slot & 4) >> 1) | (slot & 1);
-              const uint64_t qd = desc_advance(qd0, c * kChunk);
-              const uint64_t kd = qh == 2 ? rd0 : desc_advance(kd0, (s * 8 + slot) * kChunk);
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ss_2sm(d, desc_advance(qd, 32 * k), desc_advance(kd, 32 * k), idesc_qk,
-                                (qh | cc | k) != 0);
-            }
-            if (qh == 2) {
-              mma_commit_2sm_mc(bar(B_SFULL + s), 3);
-              qh = 0;
-              ++qj;
-            } else {
-              if (qh == 0) mma_commit_2sm_mc(bar(B_QH0 + s), 3);
-              ++qh;
-            }
-            prog = true;
-          }
-        }
-        if (prog) {
-          idle = 0;
-        } else if ((++idle & 255u) == 0) {
-          if (idle == 256u) t_idle = global_ns();
-          else if (global_ns() - t_idle > 1000000000ull || *abort_flag) ok = false;
-        }
+        if (*abort_flag) ok = false;
       }
       if (!ok) fail();
     }
