@@ -38,10 +38,10 @@
 // each CTA sends its rows' alpha (and whether any row needs a rescale) to the
 // peer every tile; the rescale itself is rare.
 //
-// Warp roles (256 threads): warp 0 own-token producer (+ Q), warp 1 QK issuer
-// (even CTA) and TMEM owner, warps 2-5 softmax + epilogue (TMEM lane =
-// 32*(warp%4) + lane), warp 6 peer-token producer, warp 7 PV issuer (even
-// CTA). The two issuers write disjoint TMEM (S and O^T) and each commit
+// Warp roles (384 threads): warp 0 own-token producer (+ Q), warp 1 QK issuer
+// (even CTA) and TMEM owner, warps 2-5 and 8-11 softmax + epilogue (TMEM lane
+// = 32*(warp%4) + lane; the two sets split each lane's 64 scores), warp 6
+// peer-token producer, warp 7 PV issuer (even CTA). The two issuers write disjoint TMEM (S and O^T) and each commit
 // tracks only its own thread's MMAs, so neither stream waits on the other's
 // barriers. Every wait is bounded; a timeout sets MLA_DEVICE_ERR_TIMEOUT and
 // the kernel unwinds.
@@ -57,7 +57,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kTileT = 128;                 // tokens per tile (both CTAs)
 constexpr int kChunk = 8192;                // 64 rows (tokens or query rows) x 128 B
 constexpr int kQBytes = 9 * kChunk;         // q_lat chunks 0-7, q_pe
@@ -66,7 +66,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffL = kOffQ + kQBytes;      // 2 sets x 8 latent chunk slots
 constexpr int kOffR = kOffL + 16 * kChunk;  // rope chunk slot
 constexpr int kOffP = kOffR + kChunk;       // P: 2 blocks (tokens 0-63, 64-127) of 64 rows x 128 B
-constexpr int kOffAux = kOffP + 2 * kChunk;
+constexpr int kBigBytes = kOffP + 2 * kChunk;   // the 1024-aligned operand region
 enum : int {
   B_QFULL = 0,
   B_KF0 = 1,              // [2] latent chunks 0-3 of both CTAs landed
@@ -81,16 +81,24 @@ enum : int {
   B_QH0 = 17,             // [2] QK(j) over slots 0-3 done (both CTAs, multicast)
   B_PVX = 19,             // [2] PV(j) over slots 0-3 done (both CTAs, multicast)
   B_RF = 21,              // the rope chunk of tile j of both CTAs landed (phase j)
-  B_COUNT = 22
+  B_RFREE = 22,           // QK(j) over the rope chunk done: the rope slot is free (multicast)
+  B_COUNT = 23
 };
-constexpr int kOffTmemPtr = kOffAux + 256;
+// Control block (barriers, TMEM address, abort flag, rescale flags): in the
+// alignment gap below the operand region when it fits there, else after the
+// exchange block. Exchange block (row statistics, alpha): after the operands.
+constexpr int kOffTmemPtr = 8 * B_COUNT;                  // within the control block
 constexpr int kOffAbort = kOffTmemPtr + 4;
-constexpr int kOffFlags = kOffAux + 272;    // int need[2][2]
-constexpr int kOffXmax = kOffAux + 320;     // float [128]: token-half exchange
-constexpr int kOffAlpha = kOffXmax + 512;   // float [2][128]: alpha (epilogue: output scale)
-constexpr int kSmemBytes = kOffAlpha + 1024;
-constexpr int kSmemAlloc = kSmemBytes + 1024;
-static_assert(kSmemAlloc <= 232448, "shared memory over the per-block limit");
+constexpr int kOffFlags = kOffAbort + 4;                  // int need[2][2]
+constexpr int kCtrlBytes = (kOffFlags + 16 + 15) & ~15;
+constexpr int kOffXmax = kBigBytes;                       // float [2 sets][128 lanes]
+constexpr int kOffAlpha = kOffXmax + 1024;                // float [2][128]: alpha (epilogue: output scale)
+constexpr int kXchgEnd = kOffAlpha + 1024;
+constexpr int kSmemAlloc = 232448;                        // the per-block limit
+// the base is 16-byte aligned: a gap below kCtrlBytes leaves the control
+// block after the exchange block, a larger one (at most 1008) holds it
+static_assert(kXchgEnd + kCtrlBytes + (kCtrlBytes - 16) <= kSmemAlloc, "shared memory over the per-block limit");
+static_assert(kXchgEnd + 1008 <= kSmemAlloc, "shared memory over the per-block limit");
 
 constexpr uint32_t kColS = 0;               // S buffers at columns 0 and 64 (pair M = 128 layout)
 constexpr uint32_t kColO = 128;             // O^T halves n = 0, 1 at columns 128 and 256
@@ -159,14 +167,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb0 = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sb0 - raw);
+  const uint32_t ctrl = (sb0 - raw >= (uint32_t)kCtrlBytes) ? raw : sb0 + kXchgEnd;
+  uint8_t* ctrl_p = smem_raw + (ctrl - raw);
   const DecodeParams& p = P.p;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int rb = blockIdx.x >> 1, b = blockIdx.y, z = blockIdx.z;
   pdl_launch_dependents();
-  auto bar = [&](int i) -> uint32_t { return sb0 + kOffAux + 8u * (uint32_t)i; };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  auto bar = [&](int i) -> uint32_t { return ctrl + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_p + kOffAbort);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -184,19 +194,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       mbar_init(bar(B_PVX + i), 1);
     }
     mbar_init(bar(B_RF), 1);
+    mbar_init(bar(B_RFREE), 1);
     mbar_init(bar(B_PFULL), 2);         // one arrival per CTA
     mbar_init(bar(B_EPX), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_2sm(sb0 + kOffTmemPtr, kTmemCols);
+    tmem_alloc_2sm(ctrl + kOffTmemPtr, kTmemCols);
     tmem_relinquish_2sm();
   }
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemPtr);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(ctrl_p + kOffTmemPtr);
   // the setup above overlapped the previous kernel (the absorb); global
   // inputs (q_lat, lengths, tables, the cache) are read only once it completed
   pdl_wait();
@@ -263,10 +274,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j & 1;
         prefetch_tile(j + 1);
-        // slots 0-3 of set s held tile j-2 until the first half of its aggregation
-        if (j >= 2 && !mbar_wait_cluster(bar(B_PVX + s), ((j - 2) >> 1) & 1)) { ok = false; break; }
         int y, zc;
         coords(t_begin + j * kTileT + (int)rank * 64, y, zc);
+        // the single rope slot once QK(j-1) has read it (QK takes the rope chunk
+        // first, so this load runs a latent box ahead of the tile's own boxes)
+        if (j >= 1 && !mbar_wait_cluster(bar(B_RFREE), (j - 1) & 1)) { ok = false; break; }
+        if (rank == 0) mbar_arrive_expect_tx(bar(B_RF), 2 * kChunk);
+        tma_load_3d_2sm(sb0 + kOffR, &P.tm_pe, map_to_rank(bar(B_RF), 0), 0, y, zc);
+        // slots 0-3 of set s held tile j-2 until the first half of its aggregation
+        if (j >= 2 && !mbar_wait_cluster(bar(B_PVX + s), ((j - 2) >> 1) & 1)) { ok = false; break; }
         const uint32_t dst = sb0 + kOffL + s * 8 * kChunk;
         if (rank == 0) mbar_arrive_expect_tx(bar(B_KF0 + s), 2 * 4 * kChunk);
         tma_load_5d_2sm(dst, &P.tm_kx, map_to_rank(bar(B_KF0 + s), 0), 0, y, 0, 0, zc);
@@ -274,10 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         if (j >= 2 && !mbar_wait_cluster(bar(B_PVDONE + s), ((j - 2) >> 1) & 1)) { ok = false; break; }
         if (rank == 0) mbar_arrive_expect_tx(bar(B_KF1 + s), 2 * 4 * kChunk);
         tma_load_5d_2sm(dst + 4 * kChunk, &P.tm_kx, map_to_rank(bar(B_KF1 + s), 0), 0, y, 2, 0, zc);
-        // the single rope slot once S(j-1) is computed (QK takes the rope chunk last)
-        if (j >= 1 && !mbar_wait_cluster(bar(B_SFULL + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
-        if (rank == 0) mbar_arrive_expect_tx(bar(B_RF), 2 * kChunk);
-        tma_load_3d_2sm(sb0 + kOffR, &P.tm_pe, map_to_rank(bar(B_RF), 0), 0, y, zc);
         if (*abort_flag) ok = false;
       }
       if (!ok) {
@@ -312,9 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ QK issuer (even CTA)
-    // S(j) = Q . K^T in three groups as their data lands: slots 0-3 (then a
-    // commit that frees them for the peer-token box of CTA 1), slots 4-7, the
-    // rope chunk; the S buffer must have been read by softmax(j-2).
+    // S(j) = Q . K^T in three groups as their data lands: the rope chunk (then
+    // a commit that frees the rope slot for tile j+1), slots 0-3 (then a commit
+    // that frees them for the peer-token box of CTA 1), slots 4-7; the S buffer
+    // must have been read by softmax(j-2).
     if (rank == 0 && lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       const uint64_t qd0 = smem_desc(sb0 + kOffQ, 16, 1024, kSwizzle128B);
@@ -327,24 +340,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         if (j >= 2) ok = mbar_wait_cluster(bar(B_SFREE + s), ((j - 2) >> 1) & 1);
 #pragma unroll 1
         for (int g3 = 0; g3 < 3 && ok; ++g3) {
-          ok = g3 == 2 ? mbar_wait_cluster(bar(B_RF), j & 1)
-                       : mbar_wait_cluster(bar((g3 == 0 ? B_KF0 : B_KF1) + s), (j >> 1) & 1);
+          ok = g3 == 0 ? mbar_wait_cluster(bar(B_RF), j & 1)
+                       : mbar_wait_cluster(bar((g3 == 1 ? B_KF0 : B_KF1) + s), (j >> 1) & 1);
           if (!ok) break;
           tc_fence_after();
-          const int nc = g3 == 2 ? 1 : 4;
+          const int nc = g3 == 0 ? 1 : 4;
 #pragma unroll 1
           for (int cc = 0; cc < nc; ++cc) {
-            // slot 4 g3 + cc holds latent chunk (0, 1, 4, 5, 2, 3, 6, 7)[slot]; then the rope
-            const int slot = 4 * g3 + cc;
-            const int c = g3 == 2 ? 8 : ((slot & 2) << 1) | ((slot & 4) >> 1) | (slot & 1);
+            // the rope, then slot 4 (g3 - 1) + cc holding latent chunk (0, 1, 4, 5, 2, 3, 6, 7)[slot]
+            const int slot = 4 * (g3 - 1) + cc;
+            const int c = g3 == 0 ? 8 : ((slot & 2) << 1) | ((slot & 4) >> 1) | (slot & 1);
             const uint64_t qd = desc_advance(qd0, c * kChunk);
-            const uint64_t kd = g3 == 2 ? rd0 : desc_advance(kd0, (s * 8 + slot) * kChunk);
+            const uint64_t kd = g3 == 0 ? rd0 : desc_advance(kd0, (s * 8 + slot) * kChunk);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mma_bf16_ss_2sm(d, desc_advance(qd, 32 * k), desc_advance(kd, 32 * k), idesc_qk,
                               (g3 | cc | k) != 0);
           }
-          if (g3 == 0) mma_commit_2sm_mc(bar(B_QH0 + s), 3);
+          if (g3 == 0) mma_commit_2sm_mc(bar(B_RFREE), 3);
+          if (g3 == 1) mma_commit_2sm_mc(bar(B_QH0 + s), 3);
         }
         if (ok) mma_commit_2sm_mc(bar(B_SFULL + s), 3);
         if (*abort_flag) ok = false;
@@ -388,17 +402,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    // Two warp sets read each TMEM lane quarter: set 0 (warps 2-5) takes the
+    // first 32 of the lane's 64 tokens, set 1 (warps 8-11) the last 32, so a
+    // query row's scores sit with four threads (two token halves x two sets).
     const int g = warp & 3;
+    const int sset = warp >= 8 ? 1 : 0;
     const int L = 32 * g + lane;                // TMEM lane
     const int half = L >> 6, row = L & 63;      // S: this CTA's query row, token half
-    const bool owner = half == 0;               // one thread per query row sends its stats
+    const int xi = 128 * sset + L;              // this thread's slot in the row-statistics exchange
+    const bool owner = half == 0 && sset == 0;  // one thread per query row sends its stats
     const int r = rb * 128 + (int)rank * 64 + row;
     const int q = r % p.Q;
     const int h = r / p.Q;
     const uint32_t lane_base = (uint32_t)(32 * g) << 16;
     float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
     float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
-    int* need_s = reinterpret_cast<int*>(smem + kOffFlags);
+    int* need_s = reinterpret_cast<int*>(ctrl_p + kOffFlags);
     const uint32_t peer = rank ^ 1u;
     float m_run = -INFINITY, l_part = 0.f;
     bool ab = false;
@@ -408,33 +427,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     const bool causal = p.causal != 0;
     const int causal_last = len - p.Q + q;   // last visible token of a causal row
     const bool paged = p.block_table != nullptr;
-    const bool leader_thread = (L == 0);     // arrives for this CTA on the even CTA's barriers
+    const bool leader_thread = (xi == 0);    // arrives for this CTA on the even CTA's barriers
 
     for (int j = 0; j < ntiles; ++j) {
       const int sbuf = j & 1;
-      float s[64];
+      float s[32];
       // this tile's alpha exchange: 64 rescale factors and one flag from the peer
       if (leader_thread) mbar_arrive_expect_tx(bar(B_AX + (j & 1)), 65 * 4);
       if (!ab) ab = !mbar_wait_cluster(bar(B_SFULL + sbuf), (j >> 1) & 1);
       ab = __any_sync(0xffffffffu, ab);
       if (!ab) {
         tc_fence_after();
-        uint32_t v[4][16];
+        uint32_t v[2][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_base + kColS + 64u * sbuf + 16u * c, v[c]);
+        for (int c = 0; c < 2; ++c) tmem_ld16(tmem + lane_base + kColS + 64u * sbuf + 32u * sset + 16u * c, v[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(v[c][i]);
       }
       tc_fence_before();
 
-      // scale to log2 units and mask: this thread holds tokens [tb, tb + 64);
-      // tokens [tb, tb + lim) pass the range / causal / page tests
+      // scale to log2 units and mask: this thread holds tokens [ts, ts + 32) of
+      // the 64-token block (one page) at tb; tokens [ts, ts + lim) pass the
+      // range / causal / page tests
       const int tb = t_begin + j * kTileT + 64 * half;
-      int lim = t_end - tb;
-      if (causal) lim = min(lim, causal_last - tb + 1);
+      const int ts = tb + 32 * sset;
+      int lim = t_end - ts;
+      if (causal) lim = min(lim, causal_last - ts + 1);
       if (paged && !page_ok(p, b, tb < len ? tb : 0)) lim = 0;
       if (ab) lim = 0;
       // four independent max chains (one warp per SM sub-partition: latency, not
@@ -442,43 +463,42 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (mask == nullptr) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           s[c] = (c < lim) ? s[c] * sl2 : -INFINITY;
           mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
         }
       } else {
-        // the question's mask, one byte per lane (tb is the same across the warp)
-        const uint32_t m0 = __ballot_sync(0xffffffffu, tb + lane < t_end && mask[tb + lane] != 0);
-        const uint32_t m1 = __ballot_sync(0xffffffffu, tb + 32 + lane < t_end && mask[tb + 32 + lane] != 0);
+        // the question's mask, one byte per lane (ts is the same across the warp)
+        const uint32_t m0 = __ballot_sync(0xffffffffu, ts + lane < t_end && mask[ts + lane] != 0);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool vis = c < lim && (((c < 32 ? m0 : m1) >> (c & 31)) & 1u);
+        for (int c = 0; c < 32; ++c) {
+          const bool vis = c < lim && ((m0 >> c) & 1u);
           s[c] = vis ? s[c] * sl2 : -INFINITY;
           mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
         }
       }
       float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      xmax[L] = mx;
-      // all four warps have read S(j) by now: release the buffer to the MMA
+      xmax[xi] = mx;
+      // all eight warps have read S(j) by now: release the buffer to the MMA
       // (the arrival publishes no data; tcgen05.wait::ld already returned)
-      const bool stop = bar_or(1, 128, ab);
+      const bool stop = bar_or(1, 256, ab);
       if (leader_thread) mbar_arrive_remote_relaxed(map_to_rank(bar(B_SFREE + sbuf), 0));
       if (stop) {
         ab = true;
         break;
       }
-      mx = fmaxf(mx, xmax[L ^ 64]);
+      mx = fmaxf(fmaxf(mx, xmax[xi ^ 64]), fmaxf(xmax[xi ^ 128], xmax[xi ^ 192]));
       const float m_new = fmaxf(m_run, mx);
       // the first visible score sets the reference (O^T is still zero then)
       const bool need = m_run != -INFINITY && (m_new - m_run) > kRescaleThreshold;
       float alpha = 1.f;
       if (need) alpha = exp2f(m_run - m_new);
       if (need || m_run == -INFINITY) m_run = m_new;
-      uint32_t pk[32];
+      uint32_t pk[16];
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};
       const bool none = (m_run == -INFINITY);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 16; ++c) {
         const float p0 = none ? 0.f : fast_exp2(s[2 * c] - m_run);
         const float p1 = none ? 0.f : fast_exp2(s[2 * c + 1] - m_run);
         ps4[c & 3] += p0 + p1;
@@ -494,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
         alpha_s[abuf * 128 + col] = alpha;
         st_async_b32(map_to_rank(smem_u32(alpha_s + abuf * 128 + col), peer), __float_as_uint(alpha), peer_ax);
       }
-      const bool need_cta = bar_or(1, 128, owner && need);
+      const bool need_cta = bar_or(1, 256, owner && need);
       if (leader_thread) {
         st_async_b32(map_to_rank(smem_u32(need_s + abuf * 2 + (int)rank), peer), need_cta ? 1u : 0u, peer_ax);
       }
@@ -505,17 +525,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       ab = __any_sync(0xffffffffu, ab);
       uint8_t* prow = smem + kOffP + half * kChunk + row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 val = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + 16 * (c ^ (row & 7))) = val;
+      for (int c = 0; c < 4; ++c) {
+        const uint4 val = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + 16 * ((4 * sset + c) ^ (row & 7))) = val;
       }
-      // rescale O^T columns whose row's running max moved (either CTA's rows)
+      // rescale O^T columns whose row's running max moved (either CTA's rows);
+      // set n rescales O^T half n
       const bool rescale = !ab && j > 0 && (need_cta || need_s[abuf * 2 + (int)peer] != 0);
       if (rescale) {
         tc_fence_after();
         const float* al = alpha_s + abuf * 128;
-#pragma unroll 1
-        for (int n = 0; n < 2; ++n) {
+        {
+          const int n = sset;
 #pragma unroll 1
           for (int c = 0; c < 128; c += 32) {
             uint32_t v[2][16];
@@ -536,17 +557,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      // P(j) of all four warps is written: one arrival for this CTA
-      named_bar_sync(2, 128);
+      // P(j) of all eight warps is written: one arrival for this CTA
+      named_bar_sync(2, 256);
       if (leader_thread) mbar_arrive_remote_cta(map_to_rank(bar(B_PFULL), 0));
     }
 
     // ---------------------------------------------------------------- epilogue
     // row statistics: both token halves, then each row's output scale to both CTAs
-    ab = bar_or(1, 128, ab);
-    xmax[L] = l_part;
-    named_bar_sync(2, 128);
-    const float l_tot = l_part + xmax[L ^ 64];
+    ab = bar_or(1, 256, ab);
+    xmax[xi] = l_part;
+    named_bar_sync(2, 256);
+    const float l_tot = (xmax[row] + xmax[64 + row]) + (xmax[128 + row] + xmax[192 + row]);
     float scale_o, lse;
     if (p.num_splits > 1) {
       scale_o = l_tot > 0.f ? 1.f / l_tot : 0.f;
@@ -584,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     if (ntiles > 0 && !ab) ab = !mbar_wait_cluster(bar(B_PVDONE + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1);
     if (!ab) ab = !mbar_wait_cluster(bar(B_EPX), 0);
     ab = __any_sync(0xffffffffu, ab);
-    ab = bar_or(1, 128, ab);
+    ab = bar_or(1, 256, ab);
     if (ab) fail();
     tc_fence_after();
     const bool have_o = ntiles > 0 && !ab;
@@ -597,9 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm100_kernel(const __grid_
     // lanes (L, L ^ 1); the rotation angle depends on the query index only
     const int tail0 = p.Ckv - p.rope_tail;
     const bool split = p.num_splits > 1;
-    uint8_t* stage = smem + kOffL + g * 2048;   // 16 rows x 32 dims x 4 B per warp
-#pragma unroll 1
-    for (int n = 0; n < 2; ++n) {
+    uint8_t* stage = smem + kOffL + (4 * sset + g) * 2048;   // 16 rows x 32 dims x 4 B per warp
+    {
+      const int n = sset;   // set n writes O^T half n
       const int d0 = 256 * n + 128 * (int)rank + 32 * g;   // this warp's first dim
       const int d = d0 + lane;
       const bool rot = !split && p.rope_tail > 0 && d0 + 31 >= tail0;
