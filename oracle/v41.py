@@ -8,7 +8,11 @@ Attention · latent K/V dùng chung, RoPE nửa sau và W_O nhóm":
   entry takes 288 B of K/V in the FP4 budget.
 - §2 Luồng: 64 query heads of 512 dims against the single latent, sparse
   attention with an attn_sink score column, inverse RoPE on the output, then
-  the grouped W_O (not part of this path).
+  the grouped output projection "Group-LoRA W_O (8 nhóm × 1024)" back to
+  [B, T, D_model] (``grouped_wo``);
+- §3 W_O nhóm: the output projection works per group of heads: each group
+  merges its own heads' outputs with its own small matrix, and the groups'
+  results are put side by side, instead of one large matrix.
 - §4 Profiling: FP4 latent with one E4M3 scale per 16 channels checked
   against the fp32 latent; RoPE on the tail checked by hand and undone by the
   inverse; cache bytes independent of the number of query heads.
@@ -31,9 +35,20 @@ Readings where the pages leave a step open:
   quantisation; q arrives already rotated; the output's tail is rotated back
   by the query position L_b - Q + i;
 - softmax_scale = 1/sqrt(512); the sink is a raw logit (not scaled) that
-  enters each (b,h,q) denominator once and contributes no value.
+  enters each (b,h,q) denominator once and contributes no value;
+- grouped W_O ("8 nhóm × 1024", the group shapes are garbled on the page):
+  G = 8 groups of H/G consecutive heads; group g stacks its heads' inverse-
+  rotated outputs head-major into u_g of (H/G)*512 values and applies its own
+  low-rank factor wo_a[g] (R x (H/G)*512, R = 1024) to give z_g; the z_g are
+  concatenated g-major into z of G*R values ("ghép lại"), and the shared
+  factor wo_b (D x G*R) maps z to the model width D ("phân rã", "về lại
+  [B, T, D_model]"). D_model is not on the pages (4096 is the synthetic
+  choice); without wo_b the output is z itself.
 
-Pins (tests/test_oracle_v41.py): all 256 E4M3 codes against torch's
+Pins (tests/test_oracle_v41.py): the grouped W_O against one dense matrix
+wo_b . blockdiag(wo_a[0..G-1]) on the flattened heads, one-hot inputs
+against the selected weight columns, group isolation, and the one-group
+and one-head-per-group special cases; all 256 E4M3 codes against torch's
 float8_e4m3fn conversion; the 16 E2M1 codes against the OCP MX E2M1 value
 set (tests/golden/e2m1_values.json); nearest-even ties of the quantiser;
 FP4 round-trip error bound on N(0,1) latents; 288 B per entry and cache
@@ -230,3 +245,26 @@ def shared_latent_decode(q, entries, sinks, softmax_scale, seq_lens=None, causal
     if return_all:
         return dict(x=x, attn=attn, lse=lse, latent=lat, vis=vis)
     return x
+
+
+def grouped_wo(x, wo_a, wo_b=None):
+    """Grouped low-rank output projection (4A §2 Luồng, §3 W_O nhóm).
+
+    x (B,H,Q,C) inverse-rotated attention output; wo_a (G,R,(H/G)*C): group
+    g's own factor; wo_b (D,G*R) or None. Returns (B,Q,D), or (B,Q,G*R) when
+    wo_b is None: for every (b,q), u_g = x[b, gH/G:(g+1)H/G, q, :] flattened
+    head-major, z_g = wo_a[g] u_g, z = [z_0, ..., z_{G-1}], y = wo_b z.
+    """
+    xx = np.asarray(x, F64)
+    wa = np.asarray(wo_a, F64)
+    B, H, Q, C = xx.shape
+    G, R, K = wa.shape
+    assert H % G == 0 and K == (H // G) * C
+    z = np.zeros((B, Q, G * R), F64)
+    for g in range(G):
+        heads = xx[:, g * (H // G):(g + 1) * (H // G), :, :]          # (B,H/G,Q,C)
+        u = np.transpose(heads, (0, 2, 1, 3)).reshape(B, Q, K)        # head-major
+        z[:, :, g * R:(g + 1) * R] = u @ wa[g].T
+    if wo_b is None:
+        return z
+    return z @ np.asarray(wo_b, F64).T

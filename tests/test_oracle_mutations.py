@@ -153,3 +153,37 @@ def test_append_slot_off_by_one_is_caught(monkeypatch):
         return out
     monkeypatch.setattr(mla, "cache_append", bad_cache_append)
     assert not _fp4_appends_match_cache_write(v41.fp4_cache_append)
+
+
+def test_interleaved_head_groups_are_caught(monkeypatch):
+    # heads assigned to groups round-robin (h mod G) instead of in contiguous runs
+    from test_oracle_v41 import _wo_case, wo_dense_reference
+    orig = v41.grouped_wo
+
+    def bad(x, wo_a, wo_b=None):
+        G = np.asarray(wo_a).shape[0]
+        H = np.asarray(x).shape[1]
+        perm = np.concatenate([np.arange(g, H, G) for g in range(G)])
+        return orig(np.asarray(x)[:, perm], wo_a, wo_b)
+    monkeypatch.setattr(v41, "grouped_wo", bad)
+    x, wa, wb = _wo_case(G=4)
+    assert not np.allclose(v41.grouped_wo(x, wa, wb), wo_dense_reference(x, wa, wb))
+
+
+def test_query_major_stacking_is_caught(monkeypatch):
+    # a group's heads stacked dim-major (c, h) instead of head-major (h, c)
+    from test_oracle_v41 import _wo_case, wo_dense_reference
+
+    def bad(x, wo_a, wo_b=None):
+        xx = np.asarray(x, float)
+        B, H, Q, C = xx.shape
+        wa = np.asarray(wo_a, float)
+        G, R, K = wa.shape
+        z = np.zeros((B, Q, G * R))
+        for g in range(G):
+            u = np.transpose(xx[:, g * (H // G):(g + 1) * (H // G)], (0, 2, 3, 1)).reshape(B, Q, K)
+            z[:, :, g * R:(g + 1) * R] = u @ wa[g].T
+        return z if wo_b is None else z @ np.asarray(wo_b, float).T
+    monkeypatch.setattr(v41, "grouped_wo", bad)
+    x, wa, wb = _wo_case(G=2)
+    assert not np.allclose(v41.grouped_wo(x, wa, wb), wo_dense_reference(x, wa, wb))

@@ -171,3 +171,80 @@ def test_sink_enters_split_merge_once():
 def test_e2m1_quantize_keeps_the_sign_of_a_value_rounding_to_zero():
     # a conversion rounds the magnitude and keeps the sign: -0.1 -> -0 (code 8)
     assert list(v41.e2m1_quantize(np.array([-0.1, 0.1, -0.0, 0.0]))) == [8, 0, 8, 0]
+
+
+# ----------------------------------------------------------------------------- grouped W_O
+def _wo_case(seed=0, B=2, H=8, Q=2, C=6, G=4, R=3, D=5):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((B, H, Q, C)), r.standard_normal((G, R, (H // G) * C)),
+            r.standard_normal((D, G * R)))
+
+
+def _block_diag(blocks):
+    rows = sum(b.shape[0] for b in blocks)
+    cols = sum(b.shape[1] for b in blocks)
+    out = np.zeros((rows, cols))
+    i = j = 0
+    for b in blocks:
+        out[i:i + b.shape[0], j:j + b.shape[1]] = b
+        i += b.shape[0]
+        j += b.shape[1]
+    return out
+
+
+def wo_dense_reference(x, wo_a, wo_b):
+    """The grouped factors as one dense map on the heads laid side by side."""
+    B, H, Q, C = x.shape
+    W = _block_diag(list(wo_a))                        # (G*R, H*C), group g on heads gH/G..
+    if wo_b is not None:
+        W = wo_b @ W
+    flat = np.transpose(x, (0, 2, 1, 3)).reshape(B, Q, H * C)
+    return flat @ W.T
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_grouped_wo_equals_dense_blockdiag_map(G):
+    x, wa, wb = _wo_case(G=G, R=3)
+    assert np.allclose(v41.grouped_wo(x, wa, wb), wo_dense_reference(x, wa, wb), rtol=1e-12, atol=1e-12)
+    assert np.allclose(v41.grouped_wo(x, wa), wo_dense_reference(x, wa, None), rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_wo_one_hot_selects_the_weight_column():
+    # a single nonzero x[b, h, q, c] = 1 picks column (h mod H/G)*C + c of group h // (H/G)
+    B, H, Q, C, G, R, D = 2, 8, 2, 6, 4, 3, 5
+    _, wa, wb = _wo_case(B=B, H=H, Q=Q, C=C, G=G, R=R, D=D)
+    for (b, h, q, c) in [(0, 0, 0, 0), (1, 5, 1, 4), (0, 7, 1, 5), (1, 2, 0, 3)]:
+        x = np.zeros((B, H, Q, C))
+        x[b, h, q, c] = 1.0
+        g, j = h // (H // G), h % (H // G)
+        z = np.zeros(G * R)
+        z[g * R:(g + 1) * R] = wa[g][:, j * C + c]
+        y = v41.grouped_wo(x, wa, wb)
+        others = np.ones((B, Q), bool)
+        others[b, q] = False
+        assert np.all(y[others] == 0.0)                          # exactly: no other (b, q) is touched
+        assert np.allclose(y[b, q], wb @ z, rtol=1e-14, atol=1e-14)
+        assert np.array_equal(v41.grouped_wo(x, wa)[b, q], z)   # the selected column itself
+
+
+def test_grouped_wo_groups_are_isolated():
+    x, wa, _ = _wo_case()
+    H, G, R = x.shape[1], wa.shape[0], wa.shape[1]
+    x2 = x.copy()
+    x2[:, 2 * (H // G):3 * (H // G)] += 1.0            # only group 2's heads change
+    z1, z2 = v41.grouped_wo(x, wa), v41.grouped_wo(x2, wa)
+    changed = np.any(z1 != z2, axis=(0, 1))
+    assert np.all(changed[2 * R:3 * R]) and not np.any(np.delete(changed, np.s_[2 * R:3 * R]))
+
+
+def test_grouped_wo_special_cases():
+    # one group: a plain low-rank product of the flattened heads
+    x, wa, wb = _wo_case(G=1, R=4)
+    flat = np.transpose(x, (0, 2, 1, 3)).reshape(x.shape[0], x.shape[2], -1)
+    assert np.allclose(v41.grouped_wo(x, wa, wb), (flat @ wa[0].T) @ wb.T, rtol=1e-12, atol=1e-12)
+    # one head per group: z_h = wo_a[h] x_h, per head
+    x, wa, _ = _wo_case(H=4, G=4, R=3)
+    z = v41.grouped_wo(x, wa)
+    for h in range(4):
+        assert np.allclose(z[:, :, 3 * h:3 * h + 3], np.einsum("rc,bqc->bqr", wa[h], x[:, h]),
+                           rtol=1e-12, atol=1e-12)
