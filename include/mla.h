@@ -283,6 +283,48 @@ typedef struct mla_append_args {
 
 mla_status_t mla_cache_append(const mla_append_args* a, void* stream);
 
+/*
+ * mla_group_wo - the step after the shared-latent decode's inverse RoPE: the
+ * grouped low-rank output projection (openarchlab DeepSeek-V4.1-Flash 4A,
+ * §2 Luồng "Group-LoRA W_O (8 nhóm × 1024)" back to [B, T, D_model]; §3 W_O
+ * nhóm: each group of heads has its own small projection, the groups'
+ * results side by side).
+ *
+ * For every token t = b*Q + q and group g of the G groups of H/G
+ * consecutive heads:
+ *   u_g[t]          = x[b, g*H/G .. (g+1)*H/G - 1, q, :] laid head-major ((H/G)*Ckv values)
+ *   z[t, g*R + r]   = sum_k wo_a[g, r, k] * u_g[t, k]           (group g's own factor)
+ *   out[t, n]       = sum_k wo_b[n, k] * z[t, k]                 (shared factor; omitted
+ *                                                                 when wo_b is NULL: out = z)
+ * D_model is not given by the page; D is the caller's.
+ *
+ * Layouts (row-major, bf16, device pointers owned by the caller, 16-byte
+ * aligned): x (B,H,Q,Ckv); wo_a (G,R,(H/G)*Ckv); wo_b (D,G*R) or NULL;
+ * out (B,Q,D), or (B,Q,G*R) without wo_b.
+ * Supported: q/weight dtype MLA_BF16, Ckv a multiple of 64, H a multiple of
+ *   G, R and D multiples of 128, Q in 1..16; fp32 accumulation, z rounded
+ *   to bf16 between the two factors. Anything else: MLA_ERR_UNSUPPORTED.
+ * workspace: at least mla_group_wo_workspace_size(a) bytes of device memory
+ *   (z and the split-K partial sums), or NULL when that is 0; smaller gives
+ *   MLA_ERR_WORKSPACE with nothing enqueued.
+ * err_flag: optional device int32; MLA_DEVICE_ERR_TIMEOUT when a bounded
+ *   wait inside the kernel gave up (the output is then not written).
+ */
+typedef struct mla_group_wo_args {
+  int B, H, Q, Ckv;
+  int G, R, D;             /* groups, rank per group, output width (ignored without wo_b) */
+  mla_dtype_t dtype;       /* MLA_BF16 */
+  const void* x;
+  const void* wo_a;
+  const void* wo_b;        /* or NULL */
+  void* out;
+  int32_t* err_flag;       /* optional device status word */
+} mla_group_wo_args;
+
+size_t mla_group_wo_workspace_size(const mla_group_wo_args* a);
+mla_status_t mla_group_wo(const mla_group_wo_args* a, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif

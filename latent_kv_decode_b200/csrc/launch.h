@@ -35,4 +35,9 @@ bool sm100_decode_supported(const mla_decode_args* a);
 int sm100_auto_splits(const mla_decode_args* a, int sms);
 cudaError_t launch_decode_sm100(const DecodeParams& p, const mla_decode_args* a, cudaStream_t st);
 
+// grouped low-rank output projection (tcgen05 weight-streaming GEMM with split-K):
+// bf16, Ckv % 64 == 0, H % G == 0, R and D multiples of 128, Q <= 16
+size_t group_wo_workspace_bytes(const mla_group_wo_args* a, int sms);
+cudaError_t launch_group_wo_sm100(const mla_group_wo_args* a, void* ws, int sms, cudaStream_t st);
+
 }  // namespace mla

@@ -352,3 +352,46 @@ extern "C" mla_status_t mla_cache_append(const mla_append_args* a, void* stream)
   if (s != MLA_OK) return s;
   return cuda_status(mla::launch_cache_append(a, (cudaStream_t)stream));
 }
+
+namespace {
+
+bool is_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+mla_status_t validate_group_wo(const mla_group_wo_args* a) {
+  if (!a) return MLA_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->H <= 0 || a->Q <= 0 || a->Ckv <= 0 || a->G <= 0 || a->R <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (a->wo_b && a->D <= 0) return MLA_ERR_INVALID_ARG;
+  if (!a->x || !a->wo_a || !a->out) return MLA_ERR_INVALID_ARG;
+  if (!aligned(a->x, 16) || !aligned(a->wo_a, 16) || !aligned(a->out, 16) || !aligned(a->wo_b, 16))
+    return MLA_ERR_INVALID_ARG;
+  if (a->dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
+  if (a->H % a->G != 0 || a->Ckv % 64 != 0 || a->R % 128 != 0 || a->Q > 16) return MLA_ERR_UNSUPPORTED;
+  if (a->wo_b && a->D % 128 != 0) return MLA_ERR_UNSUPPORTED;
+  // the TMA views index rows with 32-bit coordinates
+  if ((int64_t)a->B * a->H * a->Q * a->Ckv >= ((int64_t)1 << 31)) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)a->G * a->R * (a->H / a->G) * a->Ckv >= ((int64_t)1 << 31)) return MLA_ERR_UNSUPPORTED;
+  if (!is_sm100()) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t mla_group_wo_workspace_size(const mla_group_wo_args* a) {
+  if (validate_group_wo(a) != MLA_OK) return 0;
+  return mla::group_wo_workspace_bytes(a, sm_count());
+}
+
+extern "C" mla_status_t mla_group_wo(const mla_group_wo_args* a, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  mla_status_t s = validate_group_wo(a);
+  if (s != MLA_OK) return s;
+  const size_t need = mla::group_wo_workspace_bytes(a, sm_count());
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return MLA_ERR_WORKSPACE;
+  return cuda_status(mla::launch_group_wo_sm100(a, workspace, sm_count(), (cudaStream_t)stream));
+}

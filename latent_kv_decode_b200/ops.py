@@ -55,6 +55,8 @@ _SIGS = {
     "mla_combine": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "mla_decode_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "mla_cache_append": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
+    "mla_group_wo_workspace_size": (_c.c_size_t, [_c.c_void_p]),
+    "mla_group_wo": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
 }
 
 
@@ -94,6 +96,17 @@ class AppendArgs(ctypes.Structure):
         ("Lk", _c.c_int), ("seq_lens", _c.c_void_p), ("block_table", _c.c_void_p),
         ("max_pages", _c.c_int), ("page_size", _c.c_int), ("num_pages", _c.c_int),
         ("rope_tail", _c.c_int), ("rope_theta", _c.c_float), ("err_flag", _c.c_void_p),
+    ]
+
+
+class GroupWoArgs(ctypes.Structure):
+    """Mirror of ``mla_group_wo_args`` in include/mla.h (field order and types)."""
+
+    _fields_ = [
+        ("B", _c.c_int), ("H", _c.c_int), ("Q", _c.c_int), ("Ckv", _c.c_int),
+        ("G", _c.c_int), ("R", _c.c_int), ("D", _c.c_int), ("dtype", _c.c_int),
+        ("x", _c.c_void_p), ("wo_a", _c.c_void_p), ("wo_b", _c.c_void_p), ("out", _c.c_void_p),
+        ("err_flag", _c.c_void_p),
     ]
 
 
@@ -363,3 +376,50 @@ def mla_cache_append(c_kv, k_pe, kv_cache, pe_cache, seq_lens, *, stream=None, *
     """Enqueue mla_cache_append: write the new tokens into the cache in place."""
     a = make_append_args(c_kv, k_pe, kv_cache, pe_cache, seq_lens, **kw)
     _check(lib().mla_cache_append(ctypes.byref(a), _stream(stream)), "mla_cache_append")
+
+
+class GroupWoCall:
+    """Arguments and workspace of one mla_group_wo call (build once, launch many times)."""
+
+    def __init__(self, args: GroupWoArgs, out: torch.Tensor, workspace: Optional[torch.Tensor], keep):
+        self.args, self.out, self.workspace, self._keep = args, out, workspace, keep
+
+
+def make_group_wo(x: torch.Tensor, wo_a: torch.Tensor, wo_b: Optional[torch.Tensor] = None, *,
+                  out: Optional[torch.Tensor] = None, err_flag=None) -> GroupWoCall:
+    """Prepare mla_group_wo: x (B,H,Q,Ckv), wo_a (G,R,(H/G)*Ckv), wo_b (D,G*R) or None, all bf16.
+
+    Allocates ``out`` ((B,Q,D), or (B,Q,G*R) without wo_b) and the workspace
+    when not given; no GPU work.
+    """
+    _need_cuda(x, wo_a, wo_b)
+    for t in (x, wo_a, wo_b):
+        if t is not None and not t.is_contiguous():
+            raise MlaError("mla_group_wo: tensors must be contiguous")
+    B, H, Q, C = x.shape
+    G, R, _ = wo_a.shape
+    a = GroupWoArgs()
+    a.B, a.H, a.Q, a.Ckv, a.G, a.R = B, H, Q, C, G, R
+    a.D = wo_b.shape[0] if wo_b is not None else 0
+    a.dtype = _qdtype(x)
+    width = a.D if wo_b is not None else G * R
+    if out is None:
+        out = torch.empty((B, Q, width), dtype=x.dtype, device=x.device)
+    a.x, a.wo_a, a.wo_b, a.out = _ptr(x), _ptr(wo_a), _ptr(wo_b), _ptr(out)
+    a.err_flag = _ptr(err_flag)
+    need = lib().mla_group_wo_workspace_size(ctypes.byref(a))
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device) if need else None
+    return GroupWoCall(a, out, ws, (x, wo_a, wo_b, err_flag))
+
+
+def launch_group_wo(call: GroupWoCall, stream=None) -> torch.Tensor:
+    """Enqueue mla_group_wo for a prepared call; returns its output tensor."""
+    ws = call.workspace
+    _check(lib().mla_group_wo(ctypes.byref(call.args), _ptr(ws), 0 if ws is None else ws.numel(),
+                              _stream(stream)), "mla_group_wo")
+    return call.out
+
+
+def mla_group_wo(x, wo_a, wo_b=None, *, stream=None, **kw) -> torch.Tensor:
+    """Grouped low-rank output projection after the inverse RoPE -> (B,Q,D) or (B,Q,G*R)."""
+    return launch_group_wo(make_group_wo(x, wo_a, wo_b, **kw), stream=stream)

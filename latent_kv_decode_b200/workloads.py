@@ -261,6 +261,18 @@ def fp4_random_entries(B: int, Lk: int, Ckv: int = 512, seed: int = 5) -> np.nda
     return np.concatenate([codes, scales], axis=-1)
 
 
+def group_wo_inputs(B: int, H: int, Q: int, Ckv: int = 512, G: int = 8, R: int = 1024, D: int = 4096,
+                    seed: int = 6, with_wo_b: bool = True) -> dict:
+    """Inputs of the grouped output projection: x (B,H,Q,Ckv) N(0,1); wo_a
+    (G,R,(H/G)*Ckv) and wo_b (D,G*R) N(0,1)/sqrt(fan-in); all bf16-rounded."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    K1 = (H // G) * Ckv
+    out = dict(x=_store(_normal(rng, (B, H, Q, Ckv)), "bf16"),
+               wo_a=_store(_normal(rng, (G, R, K1), 1.0 / np.sqrt(K1)), "bf16"))
+    out["wo_b"] = _store(_normal(rng, (D, G * R), 1.0 / np.sqrt(G * R)), "bf16") if with_wo_b else None
+    return out
+
+
 def layout_only(name: str, seed: int) -> Workload:
     """The named workload's shapes, lengths and page table without its large
     arrays (q, caches, weights are None): for timing runs that draw those

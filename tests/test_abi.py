@@ -49,7 +49,8 @@ def test_status_strings(L):
     assert L.mla_version().decode().count(".") == 2
 
 
-@pytest.mark.parametrize("name,cls", [("mla_decode_args", "DecodeArgs"), ("mla_append_args", "AppendArgs")])
+@pytest.mark.parametrize("name,cls", [("mla_decode_args", "DecodeArgs"), ("mla_append_args", "AppendArgs"),
+                                      ("mla_group_wo_args", "GroupWoArgs")])
 def test_struct_layout_matches_header(name, cls):
     """ctypes mirror has the header's fields in the header's order."""
     from latent_kv_decode_b200 import ops
@@ -173,3 +174,25 @@ _FP4 = dict(cache_dtype=2, Dr=0, k_pe=None, pe_cache=None, kv_row_stride=288, kv
 def test_append_rejects_bad_arguments(L, over, status):
     a = _append_args(**over)
     assert L.mla_cache_append(ctypes.byref(a), None) == status
+
+
+def _group_wo_args(**over):
+    from latent_kv_decode_b200 import ops
+    a = ops.GroupWoArgs()
+    a.B, a.H, a.Q, a.Ckv, a.G, a.R, a.D, a.dtype = 32, 64, 1, 512, 8, 1024, 4096, 1
+    a.x = a.wo_a = a.wo_b = a.out = FAKE
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(x=None), 1), (dict(wo_a=None), 1), (dict(out=None), 1), (dict(B=0), 1), (dict(G=0), 1),
+    (dict(R=0), 1), (dict(D=0), 1), (dict(x=FAKE + 8), 1), (dict(wo_b=FAKE + 2), 1),
+    (dict(dtype=0), 2), (dict(G=3), 2), (dict(Ckv=96), 2), (dict(R=1000), 2), (dict(D=1000), 2),
+    (dict(Q=17), 2),
+])
+def test_group_wo_rejects_bad_arguments(L, over, status):
+    a = _group_wo_args(**over)
+    assert L.mla_group_wo(ctypes.byref(a), None, 0, None) == status
+    assert L.mla_group_wo_workspace_size(ctypes.byref(a)) == 0
