@@ -270,8 +270,11 @@ struct alignas(64) ProjTmaArgs {
   int out_cols;       // Ckv or Vd
 };
 
+// The absorb splits a head's 512 latent columns over two CTAs (blockIdx.z):
+// each loads half of the head's W_UK slice (4 chunks), so two CTAs fit on an
+// SM and all SMs get work.
 template <bool kAbsorb>
-__global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_constant__ ProjTmaArgs a) {
+__global__ void __launch_bounds__(kTThreads, 2) proj_tma_kernel(const __grid_constant__ ProjTmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb0 = (raw + 1023u) & ~1023u;
@@ -281,15 +284,17 @@ __global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_con
   const int bq = kTRows / a.Q;                    // sequences per CTA
   const int n0 = blockIdx.y * kTRows;
   const int nrows = min(kTRows, a.rows - n0);
+  constexpr int kWChunks = kAbsorb ? 4 : 8;       // weight chunks of 64 columns in this CTA
+  const int hz = kAbsorb ? (int)blockIdx.z : 0;   // absorb: latent columns [256 hz, 256 hz + 256)
 
-  // shared layout: weight chunks (8 x w_rows x 128 B) | activation chunks
+  // shared layout: weight chunks (kWChunks x w_rows x 128 B) | activation chunks
   // (a_chunks x 64 rows x 128 B) | barriers: 8 weight chunks, activations, MMAs done
   const uint32_t w_block = (uint32_t)a.w_rows * 128u;
-  const uint32_t off_a = 8u * w_block;
+  const uint32_t off_a = (uint32_t)kWChunks * w_block;
   const uint32_t off_bar = off_a + (uint32_t)a.a_chunks * (kTRows * 128u);
   auto bar = [&](int i) -> uint32_t { return sb0 + off_bar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * 10);
-  constexpr uint32_t kTmemCols = kAbsorb ? 256u : 64u;
+  constexpr uint32_t kTmemCols = kAbsorb ? 128u : 64u;
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
@@ -314,9 +319,9 @@ __global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_con
       // the weights are a read-only input: they stream in while the previous
       // kernel finishes; the activations are read only after pdl_wait()
       const int wrow = h * (a.Dn + a.Vd) + a.w_row0;
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < kWChunks; ++j) {
         mbar_arrive_expect_tx(bar(j), w_block);
-        tma_load_3d(sb0 + j * w_block, &a.tm_w, bar(j), 0, wrow, j);
+        tma_load_3d(sb0 + j * w_block, &a.tm_w, bar(j), 0, wrow, 4 * hz + j);
       }
       pdl_wait();
       mbar_arrive_expect_tx(bar(8), (uint32_t)a.a_chunks * kTRows * 128u);
@@ -327,12 +332,12 @@ __global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_con
     if (lane == 0) {
       ok = mbar_wait(bar(8), 0);
       if (kAbsorb) {
-        // D[c][n], M tile mt = latent columns [128 mt, 128 mt + 128) = weight
-        // chunks 2 mt, 2 mt + 1: A = W_UK^T (MN-major, K = the Dn rows d),
-        // B = q_nope rows (K-major)
+        // D[c][n], this CTA's M tile mt = latent columns [256 hz + 128 mt, +128)
+        // = its weight chunks 2 mt, 2 mt + 1: A = W_UK^T (MN-major, K = the Dn
+        // rows d), B = q_nope rows (K-major)
         const uint32_t idesc = idesc_bf16_f32(128, kTRows, true, false);
         const int ksteps = a.Dn >> 4;
-        for (int mt = 0; mt < 4 && ok; ++mt) {
+        for (int mt = 0; mt < 2 && ok; ++mt) {
           ok = mbar_wait(bar(2 * mt), 0) && mbar_wait(bar(2 * mt + 1), 0);
           if (!ok) break;
           tc_fence_after();
@@ -378,12 +383,11 @@ __global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_con
   const int g = warp & 3, part = warp >> 2;
   const uint32_t lane_base = (uint32_t)(32 * g) << 16;
   __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);   // weight area, free now
-  const int ocols = kAbsorb ? 512 : 128;
+  const int ocols = kAbsorb ? 256 : 128;            // this CTA's output columns
   if (done) {
-    const int ntile = kAbsorb ? 2 : 1;
-    for (int tt = 0; tt < ntile; ++tt) {
-      const int mt = kAbsorb ? part + 2 * tt : 0;
-      const int m = 128 * mt + 32 * g + lane;     // output column
+    {
+      const int mt = kAbsorb ? part : 0;
+      const int m = 128 * mt + 32 * g + lane;     // this CTA's output column
       const int c0 = kAbsorb ? 0 : 32 * part;     // absorb: a warp takes all 64 rows of its tiles
       const int c1 = kAbsorb ? kTRows : c0 + 32;
       for (int c = c0; c < c1; c += 16) {
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kTThreads, 1) proj_tma_kernel(const __grid_con
     const int upr = ocols >> 3;                   // 16-byte units per output row
     for (int e = threadIdx.x; e < nrows * upr; e += kTThreads) {
       const int n = e / upr, u = e - n * upr;
-      *reinterpret_cast<uint4*>(a.out + row_off(n0 + n, h, a.H, a.Q, a.out_cols) + u * 8) =
+      *reinterpret_cast<uint4*>(a.out + row_off(n0 + n, h, a.H, a.Q, a.out_cols) + ocols * hz + u * 8) =
           *reinterpret_cast<const uint4*>(stage + n * ocols + u * 8);
     }
   }
@@ -439,7 +443,7 @@ bool proj_encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
 size_t proj_tma_smem_bytes(bool absorb, int Dn, int Vd) {
   const int w_rows = absorb ? Dn : Vd;
   const int a_chunks = absorb ? Dn / 64 : 8;
-  return (size_t)8 * w_rows * 128 + (size_t)a_chunks * kTRows * 128 + 128 + 1024;
+  return (size_t)(absorb ? 4 : 8) * w_rows * 128 + (size_t)a_chunks * kTRows * 128 + 128 + 1024;
 }
 
 cudaError_t launch_proj_tma(bool absorb, const void* act, const void* w, void* out, int B, int H, int Q,
@@ -477,7 +481,7 @@ cudaError_t launch_proj_tma(bool absorb, const void* act, const void* w, void* o
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(H, (a.rows + kTRows - 1) / kTRows, 1);
+  cfg.gridDim = dim3(H, (a.rows + kTRows - 1) / kTRows, absorb ? 2 : 1);
   cfg.blockDim = dim3(kTThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
