@@ -19,7 +19,9 @@
  * one 512-dim latent stored as FP4 E2M1 with an E4M3 scale per 16 channels,
  * a sink logit per head, inverse RoPE on the output's last 64 dims) is the
  * openarchlab DeepSeek-V4.1-Flash page "4A · Multi-head Latent Attention"
- * (§1 Định nghĩa, §2 Luồng, §4 Profiling).
+ * (§1 Định nghĩa, §2 Luồng, §4 Profiling); the grouped output projection that
+ * follows it there (§2 Luồng, §3 W_O nhóm) is mla_group_wo. The step before
+ * the decode, writing a new token into its cache slot, is mla_cache_append.
  *
  * Conventions for every call:
  *  - Tensor pointers are DEVICE pointers owned by the caller. The library
@@ -35,8 +37,9 @@
  *    that returns anything but MLA_OK has enqueued nothing, except
  *    MLA_ERR_CUDA, which reports a failed launch (see mla_last_cuda_error).
  *  - Device pointers must be 16-byte aligned.
- *  - Supported shapes: Ckv = 512; Dr in {0 (shared-latent variant), 32, 64};
- *    Dn in {64, 128}; Vd = 128; H a multiple of 8, at most 128; Q in [1, 4].
+ *  - Supported shapes (decode, projections, combine, append): Ckv = 512; Dr
+ *    in {0 (shared-latent variant), 32, 64}; Dn in {64, 128}; Vd = 128; H a
+ *    multiple of 8, at most 128; Q in [1, 4]. mla_group_wo states its own.
  *    Anything else returns MLA_ERR_UNSUPPORTED.
  */
 #ifndef LATENT_KV_DECODE_MLA_H
