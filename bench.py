@@ -320,16 +320,17 @@ def kernel_source_hash(files) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if the
-    summary's kernel sources still hash to the value it was captured with."""
-    p = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+def profiled_traffic(workload: str, kernel: str = "decode", per: str = "launch"):
+    """DRAM bytes per launch (or per call) of a kernel from the committed ncu
+    summary profiles/<kernel>_<workload>.md, if the summary's kernel sources
+    still hash to the value it was captured with."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m_files = re.search(r"kernel sources:\s*(.+)", txt)
     m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
-    m_bytes = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", txt)
+    m_bytes = re.search(r"dram bytes per " + per + r":\s*([0-9.eE+]+)", txt)
     if not m_files or not m_hash or not m_bytes:
         return None
     files = m_files.group(1).replace("`", "").split()
@@ -586,6 +587,15 @@ def time_e2e(runner, stream, steps: int, dist=None):
 WO_GROUPS, WO_RANK, WO_DMODEL = 8, 1024, 4096   # "8 nhóm x 1024"; D_model is a synthetic choice
 
 
+def group_wo_algorithmic(B: int, H: int, Q: int, Ckv: int, G: int, R: int, D: int):
+    """Bytes and flops of one grouped W_O call: both weight factors once, x
+    read, z written and read back (bf16), y written; 2*T*(G*R*K1 + D*G*R) flops
+    for T = B*Q tokens and K1 = (H/G)*Ckv."""
+    T, K1 = B * Q, (H // G) * Ckv
+    byts = (G * R * K1 + D * G * R) * 2 + T * (H * Ckv + 2 * G * R + D) * 2
+    return byts, 2 * T * (G * R * K1 + D * G * R)
+
+
 def time_group_wo(w, dev, flush, steps: int, warmup: int, hbm: float, psrc: str):
     """The grouped W_O after the shared-latent decode (not part of the step):
     x (B,H,Q,Ckv) -> (B,Q,D) through G = 8 factors of rank 1024 and a shared
@@ -615,15 +625,15 @@ def time_group_wo(w, dev, flush, steps: int, warmup: int, hbm: float, psrc: str)
         evs[i][1].record(st)
     torch.cuda.synchronize()
     ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
-    T = w.B * w.Q
-    wbytes = (G * R * K1 + D * G * R) * 2
-    byts = wbytes + T * (w.H * w.Ckv + 2 * G * R + D) * 2      # weights, x, z out and in, y
-    flops = 2 * T * (G * R * K1 + D * G * R)
+    byts, flops = group_wo_algorithmic(w.B, w.H, w.Q, w.Ckv, G, R, D)
     ach = byts / (ms * 1e-3) / 1e9
     return {"shape": f"x ({w.B},{w.H},{w.Q},{w.Ckv}) -> G={G} x R={R} -> D={D}, bf16, fp32 accumulate",
             "ms": round(ms, 5), "steps": steps, "warmup": warmup,
             "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(ach / hbm, 4), "traffic": None, "peak_source": f"hbm_gbs of {psrc}",
+                         "frac": round(ach / hbm, 4),
+                         "traffic": profiled_traffic(w.name, kernel="group_wo", per="call"),
+                         "traffic_basis": "dram__bytes_read.sum + dram__bytes_write.sum of the two GEMM passes",
+                         "peak_source": f"hbm_gbs of {psrc}",
                          "algorithmic_bytes_per_call": int(byts), "flops_per_call": int(flops)},
             "launches_per_call": 4}
 

@@ -62,3 +62,27 @@ def test_committed_profiles_match_the_current_kernel_code():
 def test_spec_fraction_uses_the_datasheet_peak_of_the_unit():
     assert abs(bench.spec_fraction(4000.0, "GB/s") - 0.5) < 1e-12
     assert abs(bench.spec_fraction(1125.0, "TFLOP/s") - 0.5) < 1e-12
+
+
+def test_algorithmic_bytes_of_the_grouped_w_o():
+    # V4.1 shape: two 64 MiB bf16 factors, x (32, 64, 1, 512), z (32, 8192) out and back, y (32, 4096)
+    byts, flops = bench.group_wo_algorithmic(32, 64, 1, 512, 8, 1024, 4096)
+    assert byts == 2 * 64 * 2**20 + 32 * 64 * 512 * 2 + 2 * 32 * 8192 * 2 + 32 * 4096 * 2
+    assert byts == 137_625_600
+    assert flops == 2 * 32 * (8 * 1024 * 4096 + 4096 * 8192)
+
+
+def test_profiled_traffic_is_read_only_while_the_sources_match(tmp_path, monkeypatch):
+    # a summary carries the hash of the kernel code it was captured with; the
+    # bench reports its DRAM bytes only while the sources still hash to it
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "group_wo_wl.md").write_text(
+        "kernel sources: a.cu b.cuh\nkernel source hash: `0123456789abcdef` (code)\n"
+        "dram bytes per call: 1.5e8 (both passes)\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "0123456789abcdef")
+    assert bench.profiled_traffic("wl", kernel="group_wo", per="call") == 1.5e8
+    assert bench.profiled_traffic("wl", kernel="group_wo", per="launch") is None
+    assert bench.profiled_traffic("other", kernel="group_wo", per="call") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files: "fedcba9876543210")
+    assert bench.profiled_traffic("wl", kernel="group_wo", per="call") is None
